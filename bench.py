@@ -1,0 +1,319 @@
+#!/usr/bin/env python
+"""Throughput of the BigVGAN waveform decode on B200: decoded audio-seconds per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode of the 10 s stereo workload (B=2 batch items, N=400 latents -> 2 x
+320000 samples at 32 kHz, random-init weights, seeded N(0,1) latents) through the C ABI, with
+the latents already in HBM.  Audio-seconds count every batch item: B * N / 40 per step.
+
+Multi-GPU (torchrun, one process per GPU): independent replicas, each rank decoding its own
+batch with no collective on the data path ("scaling": "weak"); ranks meet only at the barriers
+around the timed region and in the max-over-ranks reduction of the timings.
+
+Timing: W untimed warm-up decodes, then K decodes, each bracketed by CUDA events on the
+launching stream; a 256 MiB buffer (> 126 MB L2) is rewritten between steps outside the events,
+so every step starts with a cold L2.  GPU clocks are sampled with nvidia-smi during the timed
+region.  `e2e` repeats the measurement through mh3a_decode_host with pinned host buffers
+(host->device copy of the latents and device->host copy of the waveform inside the timing).
+
+`--impl reference` times the fp64 CPU oracle (the correctness reference) on the host cores
+on a bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decoded audio-seconds/sec at 32 kHz on 1 B200; % of roofline per stage"
+UNIT = "audio-s/s"
+WORKLOAD = 3
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--precision", choices=["bf16x3", "fp32"], default="bf16x3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-frames", type=int, default=40,
+                    help="latent frames of one batch item the CPU baseline decodes")
+    ap.add_argument("--ref-sample-frames", type=int, default=8,
+                    help="latent frames of one batch item per reference-arm step")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampler of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def cpu_baseline(frames: int) -> dict:
+    """The oracle as it stands, on one batch item of the workload, `frames` latents."""
+    import oracle
+    from bigvgan_waveform_decoder_b200 import synthetic as S
+
+    arch, w, z = S.workload_inputs(WORKLOAD)
+    zs = z[:1, :, :frames].copy()
+    t0 = time.perf_counter()
+    oracle.decode(arch, w, zs)
+    dt = time.perf_counter() - t0
+    audio_s = frames / 40.0
+    return {"value": audio_s / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"1 batch item x {frames} latent frames ({audio_s:g} audio-s) of the "
+                      f"B=2 N=400 workload, fp64 oracle, {dt:.1f} s wall"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from bigvgan_waveform_decoder_b200 import synthetic as S
+
+    arch, w, z = S.workload_inputs(WORKLOAD)
+    zs = z[:1, :, :args.ref_sample_frames].copy()
+    audio_s = args.ref_sample_frames / 40.0
+    for _ in range(args.warmup):
+        oracle.decode(arch, w, zs)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode(arch, w, zs)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * audio_s / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "decode B=2 N=400 (10 s stereo), sampled: 1 item x "
+                               f"{args.ref_sample_frames} frames per step", "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"1 batch item x {args.ref_sample_frames} latent frames per "
+                                   "step of the B=2 N=400 workload"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from bigvgan_waveform_decoder_b200 import binding as Bd
+    from bigvgan_waveform_decoder_b200 import perfmodel as PM
+    from bigvgan_waveform_decoder_b200 import synthetic as S
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = S.WORKLOADS[WORKLOAD]
+    B, N = wl.B, wl.N
+    arch, w, _ = S.workload_inputs(WORKLOAD)
+    z = S.make_latents(B, N, arch.latent_channels, wl.seed + 1000 * rank)
+    precision = Bd.MH3A_BF16X3 if args.precision == "bf16x3" else Bd.MH3A_FP32
+    dec = Bd.Decoder(arch, w, precision=precision, max_batch=B, max_frames=N)
+    x = torch.from_numpy(z).to(dev)
+    out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
+    flush = torch.empty(FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+    audio_s = B * N / 40.0
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    dec.set_profiling(True)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        dec.decode(x, out)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    clocks = Clocks(local)
+    clocks.start()
+    launches0 = dec.launch_count()
+    step_ms, seg_sum = [], None
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        ev0.record(stream)
+        dec.decode(x, out)
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms.append(ev0.elapsed_time(ev1))
+        seg = dec.segment_times()
+        seg_sum = seg if seg_sum is None else [a + b for a, b in zip(seg_sum, seg)]
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    launches = dec.launch_count() - launches0
+    clk = clocks.stop()
+    dec.set_profiling(False)
+
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_max_ms = float(t.item())
+    value = world * args.steps * audio_s / (total_max_ms / 1e3)
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    zp = torch.from_numpy(z).pin_memory()
+    yp = torch.empty((B, 1, dec.hop * N), dtype=torch.float32).pin_memory()
+    for _ in range(args.warmup):
+        dec.decode_host(zp, yp)
+    barrier()
+    e2e_ms = []
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        ev0.record(stream)
+        dec.decode_host(zp, yp)
+        ev1.record(stream)
+        ev1.synchronize()
+        e2e_ms.append(ev0.elapsed_time(ev1))
+    t = torch.tensor([sum(e2e_ms)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * args.steps * audio_s / (float(t.item()) / 1e3)
+
+    # per-segment roofline
+    tc_stages = tuple(i for i in range(arch.n_stages) if precision == Bd.MH3A_BF16X3)
+    segs = PM.segments(arch, B, N, tc_stages=())
+    peaks = PM.measured_peaks()
+    p_fp32 = PM.fp32_peak_tflops(peaks["sm_max_mhz"])
+    p_tc = peaks["bf16_tflops"] / 3.0
+    seg_ms = [s / args.steps for s in (seg_sum or [])]
+    stages = []
+    for sgm, ms in zip(segs, seg_ms):
+        roof = PM.roofline_time(sgm, p_tc, p_fp32, peaks["hbm_gbs"]) * 1e3
+        stages.append({"segment": sgm.name, "ms": round(ms, 4), "roof_ms": round(roof, 4),
+                       "frac": round(roof / ms, 4) if ms > 0 else None,
+                       "tflops": round(sgm.flops / (ms * 1e-3) / 1e12, 2) if ms > 0 else None,
+                       "pipe": "tensor" if sgm.tensor else "fp32"})
+    dom = max(range(len(stages)), key=lambda i: stages[i]["ms"]) if stages else None
+    roofline = None
+    if dom is not None:
+        sgm, ms = segs[dom], seg_ms[dom]
+        launches_in_seg = 6 if sgm.name.startswith("amp") else 1
+        if sgm.tensor:
+            achieved = sgm.conv_flops / (ms * 1e-3) / 1e12
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
+                        "frac": achieved / p_tc, "traffic": None,
+                        "kernel": f"{sgm.name} conv (3 residual blocks per launch)",
+                        "launches_per_step": launches_in_seg,
+                        "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
+                                      "bf16 products per fp32 product"}
+        else:
+            achieved = sgm.flops / (ms * 1e-3) / 1e12
+            roofline = {"bound": "alu", "achieved": achieved, "peak": p_fp32, "unit": "TFLOP/s",
+                        "frac": achieved / p_fp32, "traffic": None,
+                        "kernel": f"{sgm.name} fp32 conv+activation (3 residual blocks per launch)",
+                        "launches_per_step": launches_in_seg,
+                        "peak_basis": f"148 SM x 128 fp32 lanes x 2 x {peaks['sm_max_mhz']} MHz"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16x3" if precision == Bd.MH3A_BF16X3 else "f32",
+        "data": "synthetic",
+        "config": {"workload": f"decode B={B} N={N} (10 s stereo, 2 x 320000 samples) per GPU",
+                   "global_batch": B * world, "latent_frames": N, "replicas": world,
+                   "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)"},
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": int(z.nbytes), "d2h_bytes_per_step": int(yp.numel() * 4)},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "stages": stages,
+        "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16x3_tflops": p_tc, "fp32_tflops": p_fp32,
+                  "source": peaks["source"]},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample_frames)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

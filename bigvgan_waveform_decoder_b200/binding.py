@@ -1,0 +1,249 @@
+"""Thin ctypes binding of the C ABI in include/mh3a.h (argument marshalling only).
+
+Every step of the decode runs in the CUDA library ``libmh3a.so`` built in this package
+directory; there is no fallback.  If the library is missing or cannot be loaded, every call
+raises ``RuntimeError``.  PyTorch is used only for device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmh3a.so")
+
+MH3A_FP32 = 0
+MH3A_BF16X3 = 1
+MH3A_FLAG_NO_CLAMP = 1
+MAX_STAGES, MAX_RESBLOCKS, MAX_DILATIONS = 8, 4, 4
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "shape mismatch",
+          4: "missing weight", 5: "allocation failed", 6: "CUDA error", 7: "unsupported request"}
+
+EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_decode", "mh3a_decode_host",
+           "mh3a_amp_stage", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
+           "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error")
+
+
+class mh3a_config(C.Structure):
+    _fields_ = [
+        ("latent_channels", C.c_int),
+        ("latent_dim", C.c_int),
+        ("decoder_dim", C.c_int),
+        ("n_stages", C.c_int),
+        ("rates", C.c_int * MAX_STAGES),
+        ("kernels", C.c_int * MAX_STAGES),
+        ("n_resblocks", C.c_int),
+        ("rb_kernels", C.c_int * MAX_RESBLOCKS),
+        ("n_dilations", C.c_int),
+        ("rb_dilations", (C.c_int * MAX_DILATIONS) * MAX_RESBLOCKS),
+        ("sampling_rate", C.c_int),
+        ("precision", C.c_int),
+        ("flags", C.c_uint),
+        ("latents_mean", C.POINTER(C.c_float)),
+        ("latents_std", C.POINTER(C.c_float)),
+        ("max_batch", C.c_int),
+        ("max_frames", C.c_int),
+    ]
+
+
+class mh3a_tensor(C.Structure):
+    _fields_ = [
+        ("name", C.c_char_p),
+        ("host_data", C.POINTER(C.c_float)),
+        ("ndim", C.c_int),
+        ("shape", C.c_longlong * 3),
+    ]
+
+
+class MH3AError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        msg = f"{what}: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def load():
+    """Load libmh3a.so (once).  Raises RuntimeError when it is absent: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                           "(run python -m bigvgan_waveform_decoder_b200.build)")
+    L = C.CDLL(LIB_PATH)
+    vp = C.c_void_p
+    L.mh3a_default_config.argtypes = [C.POINTER(mh3a_config)]
+    L.mh3a_default_config.restype = None
+    L.mh3a_create.argtypes = [C.POINTER(mh3a_config), C.POINTER(mh3a_tensor), C.c_int, C.POINTER(vp)]
+    L.mh3a_create.restype = C.c_int
+    L.mh3a_decode.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
+    L.mh3a_decode.restype = C.c_int
+    L.mh3a_decode_host.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
+    L.mh3a_decode_host.restype = C.c_int
+    L.mh3a_amp_stage.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, vp, vp]
+    L.mh3a_amp_stage.restype = C.c_int
+    L.mh3a_set_profiling.argtypes = [vp, C.c_int]
+    L.mh3a_set_profiling.restype = C.c_int
+    L.mh3a_segment_times.argtypes = [vp, C.POINTER(C.c_float), C.c_int, C.POINTER(C.c_int)]
+    L.mh3a_segment_times.restype = C.c_int
+    L.mh3a_launch_count.argtypes = [vp]
+    L.mh3a_launch_count.restype = C.c_longlong
+    L.mh3a_device_bytes.argtypes = [vp]
+    L.mh3a_device_bytes.restype = C.c_longlong
+    L.mh3a_destroy.argtypes = [vp]
+    L.mh3a_destroy.restype = None
+    L.mh3a_status_string.argtypes = [C.c_int]
+    L.mh3a_status_string.restype = C.c_char_p
+    L.mh3a_last_error.argtypes = []
+    L.mh3a_last_error.restype = C.c_char_p
+    _lib = L
+    return L
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        detail = load().mh3a_last_error().decode() if st == 6 else ""
+        raise MH3AError(st, what, detail)
+
+
+def make_config(arch, precision: int = MH3A_BF16X3, max_batch: int = 2, max_frames: int = 400,
+                no_clamp: bool = False):
+    """mh3a_config from an architecture object with the fields of synthetic.Arch.
+    Returns (config, keepalive)."""
+    cfg = mh3a_config()
+    load().mh3a_default_config(C.byref(cfg))
+    cfg.latent_channels = arch.latent_channels
+    cfg.latent_dim = arch.latent_dim
+    cfg.decoder_dim = arch.decoder_dim
+    cfg.n_stages = len(arch.rates)
+    for i, (r, k) in enumerate(zip(arch.rates, arch.kernels)):
+        cfg.rates[i] = r
+        cfg.kernels[i] = k
+    cfg.n_resblocks = len(arch.rb_kernels)
+    for j, k in enumerate(arch.rb_kernels):
+        cfg.rb_kernels[j] = k
+    cfg.n_dilations = len(arch.rb_dilations[0])
+    for j, ds in enumerate(arch.rb_dilations):
+        for m, d in enumerate(ds):
+            cfg.rb_dilations[j][m] = d
+    cfg.precision = precision
+    cfg.flags = MH3A_FLAG_NO_CLAMP if no_clamp else 0
+    cfg.max_batch = max_batch
+    cfg.max_frames = max_frames
+    keep = []
+    if getattr(arch, "latents_mean", None) is not None:
+        m = np.ascontiguousarray(arch.latents_mean, dtype=np.float32)
+        keep.append(m)
+        cfg.latents_mean = m.ctypes.data_as(C.POINTER(C.c_float))
+    if getattr(arch, "latents_std", None) is not None:
+        s = np.ascontiguousarray(arch.latents_std, dtype=np.float32)
+        keep.append(s)
+        cfg.latents_std = s.ctypes.data_as(C.POINTER(C.c_float))
+    return cfg, keep
+
+
+def make_table(weights: dict):
+    keep = []
+    arr = (mh3a_tensor * len(weights))()
+    for i, (name, a) in enumerate(weights.items()):
+        a = np.ascontiguousarray(a, dtype=np.float32)
+        nb = name.encode()
+        keep += [a, nb]
+        arr[i].name = nb
+        arr[i].host_data = a.ctypes.data_as(C.POINTER(C.c_float))
+        arr[i].ndim = a.ndim
+        for d in range(3):
+            arr[i].shape[d] = a.shape[d] if d < a.ndim else 1
+    return arr, keep
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+class Decoder:
+    """Owns one mh3a handle on the current CUDA device."""
+
+    def __init__(self, arch, weights: dict, precision: int = MH3A_BF16X3, max_batch: int = 2,
+                 max_frames: int = 400, no_clamp: bool = False):
+        L = load()
+        self.arch = arch
+        self.hop = int(np.prod(arch.rates))
+        self.latent_channels = arch.latent_channels
+        cfg, keep = make_config(arch, precision, max_batch, max_frames, no_clamp)
+        tab, keep2 = make_table(weights)
+        h = C.c_void_p()
+        _check(L.mh3a_create(C.byref(cfg), tab, len(weights), C.byref(h)), "mh3a_create")
+        self._h = h
+        del keep, keep2
+
+    @property
+    def handle(self):
+        return self._h
+
+    def decode(self, latents, out=None, stream=None):
+        """latents: CUDA float32 tensor [B, 32, N] -> CUDA float32 [B, 1, hop*N]."""
+        import torch
+        assert latents.is_cuda and latents.dtype == torch.float32 and latents.is_contiguous()
+        B, _, N = latents.shape
+        if out is None:
+            out = torch.empty((B, 1, self.hop * N), device=latents.device, dtype=torch.float32)
+        _check(load().mh3a_decode(self._h, latents.data_ptr(), B, N, out.data_ptr(),
+                                  _stream_ptr(stream)), "mh3a_decode")
+        return out
+
+    def decode_host(self, latents, out, stream=None):
+        """Host (ideally pinned) float32 tensors or arrays; blocks until `out` is filled."""
+        B, _, N = latents.shape
+        lp = latents.data_ptr() if hasattr(latents, "data_ptr") else latents.ctypes.data
+        op = out.data_ptr() if hasattr(out, "data_ptr") else out.ctypes.data
+        _check(load().mh3a_decode_host(self._h, lp, B, N, op, _stream_ptr(stream)),
+               "mh3a_decode_host")
+        return out
+
+    def amp_stage(self, x, stage: int, out=None, stream=None):
+        import torch
+        assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+        B, _, Lx = x.shape
+        if out is None:
+            out = torch.empty_like(x)
+        _check(load().mh3a_amp_stage(self._h, x.data_ptr(), B, Lx, stage, out.data_ptr(),
+                                     _stream_ptr(stream)), "mh3a_amp_stage")
+        return out
+
+    def set_profiling(self, on: bool):
+        _check(load().mh3a_set_profiling(self._h, 1 if on else 0), "mh3a_set_profiling")
+
+    def segment_times(self):
+        buf = (C.c_float * 64)()
+        n = C.c_int()
+        _check(load().mh3a_segment_times(self._h, buf, 64, C.byref(n)), "mh3a_segment_times")
+        return [buf[i] for i in range(n.value)]
+
+    def launch_count(self) -> int:
+        return int(load().mh3a_launch_count(self._h))
+
+    def device_bytes(self) -> int:
+        return int(load().mh3a_device_bytes(self._h))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load().mh3a_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,665 @@
+// mh3a_api.cu -- the C ABI (include/mh3a.h): configuration checks, weight folding at create
+// time, workspace management and the launch sequence of the decode.
+//
+// Decode (FastVideo "minimax_h3_audio_vae" page, `MLXMiniMaxH3AudioVAE.decode`):
+//   h = conv1x1(z) (dec_in_proj)  ->  h = conv_k7(h) (conv_pre, weight-normed, padding 3)
+//   for each stage i: h = convT(h; r_i, K_i, padding (K_i - r_i)/2)   (ups.i.0)
+//                     h = mean_j AMP_j(h)                           (resblocks 3i + j)
+//   h = act(h) (activation_post)  ->  y = conv_k7(h) (conv_post)  ->  clamp(y, -1, 1)
+// AMP_j(x): for each dilation d: x = x + conv_k,1(act(conv_k,d(act(x)))), k = rb_kernels[j].
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "mh3a_internal.cuh"
+#include "tc_kernels.cuh"
+
+using namespace mh3a;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+mh3a_status cuda_fail(cudaError_t e, const char* what) {
+    g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return MH3A_ERR_CUDA;
+}
+
+#define CK_CUDA(call, what)                                  \
+    do {                                                     \
+        cudaError_t e_ = (call);                             \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what);   \
+    } while (0)
+
+constexpr int kMaxSegments = 2 + 2 * MH3A_MAX_STAGES + 1;
+
+// Kaiser-windowed sinc low-pass of the activation (FastVideo "minimax_h3_audio_vae" page,
+// `kaiser_sinc_filter1d`): Kaiser's estimate A = 2.285 (K/2 - 1) pi (4 hw) + 7.95 of the stop-band
+// attenuation, his rule for the window shape beta(A), a symmetric Kaiser window over K points,
+// a sinc of cutoff fc on the half-integer (even K) grid, and unit DC gain.
+double bessel0(double x) {
+    // I0(x) = sum_n ((x/2)^n / n!)^2
+    double half = 0.5 * x, term = 1.0, total = 1.0;
+    for (int n = 1; n < 300 && term > 1e-20 * total; ++n) {
+        term *= (half / n) * (half / n);
+        total += term;
+    }
+    return total;
+}
+
+void build_filter(ActFilter* f) {
+    const int K = kFilterTaps;
+    const double fc = 0.5 / 2.0, hw = 0.6 / 2.0;  // ratio 2
+    const double A = 2.285 * (K / 2 - 1) * M_PI * (4.0 * hw) + 7.95;
+    const double beta = (A > 50.0) ? 0.1102 * (A - 8.7)
+                      : (A >= 21.0) ? 0.5842 * std::pow(A - 21.0, 0.4) + 0.07886 * (A - 21.0)
+                                    : 0.0;
+    double h[K], total = 0.0;
+    for (int n = 0; n < K; ++n) {
+        const double pos = (n - (K - 1) / 2.0) / ((K - 1) / 2.0);  // -1 .. 1
+        const double win = bessel0(beta * std::sqrt(std::max(0.0, 1.0 - pos * pos))) / bessel0(beta);
+        const double t = n - K / 2 + ((K % 2 == 0) ? 0.5 : 0.0);
+        const double x = 2.0 * fc * t;
+        const double sinc = (x == 0.0) ? 1.0 : std::sin(M_PI * x) / (M_PI * x);
+        h[n] = 2.0 * fc * win * sinc;
+        total += h[n];
+    }
+    for (int n = 0; n < K; ++n) {
+        f->down[n] = (float)(h[n] / total);
+        f->up[n] = 2.0f * f->down[n];  // upsampler gain = ratio
+    }
+}
+
+struct Lookup {
+    const mh3a_tensor* w;
+    int n;
+    const mh3a_tensor* find(const std::string& name) const {
+        for (int i = 0; i < n; ++i)
+            if (w[i].name && name == w[i].name) return &w[i];
+        return nullptr;
+    }
+};
+
+long long numel(const mh3a_tensor* t) {
+    long long n = 1;
+    for (int d = 0; d < t->ndim; ++d) n *= t->shape[d];
+    return n;
+}
+
+}  // namespace
+
+struct mh3a_handle {
+    mh3a_config cfg{};
+    int device = 0;
+    int hop = 1;
+    ActFilter filt{};
+    // fp32 weights (weight norm folded), [Cin, K, Cout]
+    DevConv in_proj, pre, ups[MH3A_MAX_STAGES], post;
+    DevConv rb1[MH3A_MAX_STAGES][MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS];
+    DevConv rb2[MH3A_MAX_STAGES][MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS];
+    DevAct act1[MH3A_MAX_STAGES][MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS];
+    DevAct act2[MH3A_MAX_STAGES][MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS];
+    DevAct act_post;
+    TcStageWeights tc[MH3A_MAX_STAGES];   // tensor-core operand copies (BF16X3)
+    bool stage_tc[MH3A_MAX_STAGES] = {};
+    char* warena = nullptr;
+    size_t wbytes = 0;
+    // workspace
+    char* arena = nullptr;
+    size_t abytes = 0;
+    long long stage_cap = 0;   // floats per stage buffer
+    float* buf_in = nullptr;   // [B, latent_dim, N]
+    float* buf_pre = nullptr;  // [B, decoder_dim, N]
+    float* H = nullptr;
+    float* X[MH3A_MAX_RESBLOCKS] = {};
+    float* T[MH3A_MAX_RESBLOCKS] = {};
+    float* lat_io = nullptr;   // host-API staging
+    float* wav_io = nullptr;
+    // profiling
+    bool profiling = false;
+    cudaEvent_t ev[kMaxSegments + 1] = {};
+    int nseg = 0;
+    long long launches = 0;
+};
+
+namespace {
+
+int stage_channels(const mh3a_config& c, int i) { return c.decoder_dim >> (i + 1); }
+
+mh3a_status validate(const mh3a_config& c) {
+    if (c.n_stages < 1 || c.n_stages > MH3A_MAX_STAGES) return MH3A_ERR_CONFIG;
+    if (c.n_resblocks < 1 || c.n_resblocks > MH3A_MAX_RESBLOCKS) return MH3A_ERR_CONFIG;
+    if (c.n_dilations < 1 || c.n_dilations > MH3A_MAX_DILATIONS) return MH3A_ERR_CONFIG;
+    if (c.latent_channels < 1 || c.latent_dim < 1 || c.decoder_dim < 1) return MH3A_ERR_CONFIG;
+    long long hop = 1;
+    for (int i = 0; i < c.n_stages; ++i) {
+        const int r = c.rates[i], K = c.kernels[i];
+        if (r < 1 || r > 8 || K < r || (K - r) % 2 != 0) return MH3A_ERR_CONFIG;
+        hop *= r;
+    }
+    if (hop != 800) return MH3A_ERR_CONFIG;
+    if (c.decoder_dim % (1 << c.n_stages) != 0) return MH3A_ERR_CONFIG;
+    for (int j = 0; j < c.n_resblocks; ++j) {
+        const int k = c.rb_kernels[j];
+        if (k < 1 || k % 2 == 0 || k > 31) return MH3A_ERR_CONFIG;
+        for (int m = 0; m < c.n_dilations; ++m)
+            if (c.rb_dilations[j][m] < 1 || c.rb_dilations[j][m] > 16) return MH3A_ERR_CONFIG;
+    }
+    if (c.precision != MH3A_FP32 && c.precision != MH3A_BF16X3) return MH3A_ERR_CONFIG;
+    if (c.max_batch < 1 || c.max_frames < 1) return MH3A_ERR_CONFIG;
+    return MH3A_OK;
+}
+
+// Host staging of the folded weights before one device copy.
+struct HostArena {
+    std::vector<float> data;
+    struct Fix { float** dst; size_t off; };
+    std::vector<Fix> fix;
+    size_t add(const std::vector<float>& v, float** dst) {
+        size_t off = data.size();
+        data.insert(data.end(), v.begin(), v.end());
+        data.resize((data.size() + 63) & ~size_t(63), 0.f);  // 256-byte alignment of the next
+        fix.push_back({dst, off});
+        return off;
+    }
+};
+
+// Weight-normed conv [O, I, K] -> folded, transposed to [I, K, O].
+mh3a_status fold_conv(const Lookup& lk, const std::string& prefix, int O, int I, int K, bool bias_required,
+                      HostArena& ha, DevConv* dc, std::vector<float>* folded_oik = nullptr) {
+    const mh3a_tensor* v = lk.find(prefix + ".weight_v");
+    const mh3a_tensor* g = lk.find(prefix + ".weight_g");
+    if (!v || !g) return MH3A_ERR_MISSING_WEIGHT;
+    if (!v->host_data || !g->host_data) return MH3A_ERR_INVALID_ARG;
+    if (v->ndim != 3 || v->shape[0] != O || v->shape[1] != I || v->shape[2] != K || numel(g) != O)
+        return MH3A_ERR_SHAPE;
+    std::vector<float> w((size_t)I * K * O);
+    if (folded_oik) folded_oik->assign((size_t)O * I * K, 0.f);
+    for (int o = 0; o < O; ++o) {
+        const float* vo = v->host_data + (size_t)o * I * K;
+        double ss = 0.0;
+        for (long long q = 0; q < (long long)I * K; ++q) ss += (double)vo[q] * vo[q];
+        const double sc = (double)g->host_data[o] / std::sqrt(ss);
+        for (int c = 0; c < I; ++c)
+            for (int j = 0; j < K; ++j) {
+                const float val = (float)(sc * vo[(size_t)c * K + j]);
+                w[((size_t)c * K + j) * O + o] = val;
+                if (folded_oik) (*folded_oik)[((size_t)o * I + c) * K + j] = val;
+            }
+    }
+    ha.add(w, &dc->w);
+    const mh3a_tensor* b = lk.find(prefix + ".bias");
+    if (b) {
+        if (numel(b) != O) return MH3A_ERR_SHAPE;
+        ha.add(std::vector<float>(b->host_data, b->host_data + O), &dc->b);
+    } else if (bias_required) {
+        return MH3A_ERR_MISSING_WEIGHT;
+    } else {
+        ha.add(std::vector<float>(O, 0.f), &dc->b);
+    }
+    dc->cin = I;
+    dc->cout = O;
+    dc->k = K;
+    return MH3A_OK;
+}
+
+// Weight-normed transposed conv [I, O, K] (norm per input channel) -> [I, K, O].
+mh3a_status fold_convT(const Lookup& lk, const std::string& prefix, int I, int O, int K, HostArena& ha,
+                       DevConv* dc) {
+    const mh3a_tensor* v = lk.find(prefix + ".weight_v");
+    const mh3a_tensor* g = lk.find(prefix + ".weight_g");
+    const mh3a_tensor* b = lk.find(prefix + ".bias");
+    if (!v || !g || !b) return MH3A_ERR_MISSING_WEIGHT;
+    if (v->ndim != 3 || v->shape[0] != I || v->shape[1] != O || v->shape[2] != K || numel(g) != I ||
+        numel(b) != O)
+        return MH3A_ERR_SHAPE;
+    std::vector<float> w((size_t)I * K * O);
+    for (int c = 0; c < I; ++c) {
+        const float* vc = v->host_data + (size_t)c * O * K;
+        double ss = 0.0;
+        for (long long q = 0; q < (long long)O * K; ++q) ss += (double)vc[q] * vc[q];
+        const double sc = (double)g->host_data[c] / std::sqrt(ss);
+        for (int o = 0; o < O; ++o)
+            for (int j = 0; j < K; ++j) w[((size_t)c * K + j) * O + o] = (float)(sc * vc[(size_t)o * K + j]);
+    }
+    ha.add(w, &dc->w);
+    ha.add(std::vector<float>(b->host_data, b->host_data + O), &dc->b);
+    dc->cin = I;
+    dc->cout = O;
+    dc->k = K;
+    return MH3A_OK;
+}
+
+mh3a_status load_act(const Lookup& lk, const std::string& prefix, int C, HostArena& ha, DevAct* da) {
+    const mh3a_tensor* a = lk.find(prefix + ".alpha");
+    const mh3a_tensor* b = lk.find(prefix + ".beta");
+    if (!a || !b) return MH3A_ERR_MISSING_WEIGHT;
+    if (numel(a) != C || numel(b) != C) return MH3A_ERR_SHAPE;
+    std::vector<float> ib(C);
+    for (int c = 0; c < C; ++c) ib[c] = (float)(1.0 / ((double)b->host_data[c] + 1e-9));
+    ha.add(std::vector<float>(a->host_data, a->host_data + C), &da->alpha);
+    ha.add(ib, &da->inv_beta);
+    return MH3A_OK;
+}
+
+mh3a_status record(mh3a_handle* h, cudaStream_t s) {
+    if (!h->profiling) return MH3A_OK;
+    if (h->nseg > kMaxSegments) return MH3A_OK;
+    CK_CUDA(cudaEventRecord(h->ev[h->nseg], s), "cudaEventRecord");
+    h->nseg++;
+    return MH3A_OK;
+}
+
+mh3a_status counted(mh3a_handle* h, int n) {
+    if (n < 0) {
+        cudaError_t e = cudaGetLastError();
+        return cuda_fail(e == cudaSuccess ? cudaErrorLaunchFailure : e, "kernel launch");
+    }
+    h->launches += n;
+    return MH3A_OK;
+}
+
+// The six residual-chain launches of one AMP stage: input h (B, C, L); the per-block running
+// sums end in h->X[j].  Every launch covers all residual blocks (blockIdx.z).
+mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cudaStream_t s) {
+    const mh3a_config& c = h->cfg;
+    const int C = stage_channels(c, stage);
+    const int nrb = c.n_resblocks;
+    for (int m = 0; m < c.n_dilations; ++m) {
+        for (int half = 0; half < 2; ++half) {
+            ConvParams p{};
+            p.Cin = C;
+            p.Cout = C;
+            p.L = L;
+            p.B = B;
+            p.clamp = 0;
+            p.filt = h->filt;
+            for (int j = 0; j < nrb; ++j) {
+                const int k = c.rb_kernels[j];
+                const int d = (half == 0) ? c.rb_dilations[j][m] : 1;
+                ConvJob& J = p.job[j];
+                const DevConv& dc = (half == 0) ? h->rb1[stage][j][m] : h->rb2[stage][j][m];
+                const DevAct& da = (half == 0) ? h->act1[stage][j][m] : h->act2[stage][j][m];
+                J.x0 = (half == 0) ? (m == 0 ? in : h->X[j]) : h->T[j];
+                J.w = dc.w;
+                J.bias = dc.b;
+                J.alpha = da.alpha;
+                J.inv_beta = da.inv_beta;
+                J.res = (half == 0) ? nullptr : (m == 0 ? in : h->X[j]);
+                J.out = (half == 0) ? h->T[j] : h->X[j];
+                J.K = k;
+                J.dil = d;
+                J.pad = d * (k - 1) / 2;
+            }
+            int n;
+            if (h->stage_tc[stage])
+                n = launch_conv_tc(p, nrb, h->tc[stage], m, half, s);
+            else
+                n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
+            mh3a_status st = counted(h, n);
+            if (st) return st;
+        }
+    }
+    return MH3A_OK;
+}
+
+mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* out, cudaStream_t s) {
+    const mh3a_config& c = h->cfg;
+    h->nseg = 0;
+    mh3a_status st = record(h, s);
+    if (st) return st;
+    // dec_in_proj (denormalisation folded in)
+    {
+        ConvParams p{};
+        p.Cin = c.latent_channels;
+        p.Cout = c.latent_dim;
+        p.L = N;
+        p.B = B;
+        p.job[0].x0 = lat;
+        p.job[0].w = h->in_proj.w;
+        p.job[0].bias = h->in_proj.b;
+        p.job[0].out = h->buf_in;
+        p.job[0].K = 1;
+        p.job[0].dil = 1;
+        p.job[0].pad = 0;
+        if ((st = counted(h, launch_conv_simt(p, 1, false, false, s)))) return st;
+        if ((st = record(h, s))) return st;
+    }
+    // conv_pre
+    {
+        ConvParams p{};
+        p.Cin = c.latent_dim;
+        p.Cout = c.decoder_dim;
+        p.L = N;
+        p.B = B;
+        p.job[0].x0 = h->buf_in;
+        p.job[0].w = h->pre.w;
+        p.job[0].bias = h->pre.b;
+        p.job[0].out = h->buf_pre;
+        p.job[0].K = h->pre.k;
+        p.job[0].dil = 1;
+        p.job[0].pad = 3;
+        int n = h->stage_tc[0] ? launch_conv_pre_tc(p, h->tc[0], s) : launch_conv_simt(p, 1, false, false, s);
+        if ((st = counted(h, n))) return st;
+        if ((st = record(h, s))) return st;
+    }
+    int C = c.decoder_dim, L = N;
+    for (int i = 0; i < c.n_stages; ++i) {
+        ConvTParams q{};
+        const bool mean3 = (i > 0);
+        q.x0 = (i == 0) ? h->buf_pre : h->X[0];
+        q.x1 = mean3 ? h->X[1] : nullptr;
+        q.x2 = mean3 ? h->X[2] : nullptr;
+        q.w = h->ups[i].w;
+        q.bias = h->ups[i].b;
+        q.out = h->H;
+        q.Cin = C;
+        q.Cout = C / 2;
+        q.Lin = L;
+        q.B = B;
+        q.r = c.rates[i];
+        q.K = c.kernels[i];
+        q.pad = (q.K - q.r) / 2;
+        if (mean3 && c.n_resblocks != 3) {
+            // the fused mean reads exactly three block outputs; otherwise reduce explicitly
+            return MH3A_ERR_UNSUPPORTED;
+        }
+        if ((st = counted(h, launch_convT_simt(q, mean3, s)))) return st;
+        if ((st = record(h, s))) return st;
+        C /= 2;
+        L *= c.rates[i];
+        if ((st = run_amp(h, i, h->H, B, L, s))) return st;
+        if ((st = record(h, s))) return st;
+    }
+    // activation_post + conv_post + clamp, reading the mean of the last stage's blocks
+    {
+        ConvParams p{};
+        p.Cin = C;
+        p.Cout = 1;
+        p.L = L;
+        p.B = B;
+        p.clamp = (c.flags & MH3A_FLAG_NO_CLAMP) ? 0 : 1;
+        p.filt = h->filt;
+        p.job[0].x0 = h->X[0];
+        p.job[0].x1 = h->X[1];
+        p.job[0].x2 = h->X[2];
+        p.job[0].w = h->post.w;
+        p.job[0].bias = h->post.b;
+        p.job[0].alpha = h->act_post.alpha;
+        p.job[0].inv_beta = h->act_post.inv_beta;
+        p.job[0].out = out;
+        p.job[0].K = h->post.k;
+        p.job[0].dil = 1;
+        p.job[0].pad = 3;
+        if ((st = counted(h, launch_conv_simt(p, 1, true, true, s)))) return st;
+        if ((st = record(h, s))) return st;
+    }
+    return MH3A_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void mh3a_default_config(mh3a_config* c) {
+    if (!c) return;
+    std::memset(c, 0, sizeof(*c));
+    c->latent_channels = 32;
+    c->latent_dim = 2048;
+    c->decoder_dim = 1024;
+    c->n_stages = 7;
+    const int rates[7] = {5, 5, 2, 2, 2, 2, 2}, kernels[7] = {9, 9, 4, 4, 4, 4, 4};
+    for (int i = 0; i < 7; ++i) {
+        c->rates[i] = rates[i];
+        c->kernels[i] = kernels[i];
+    }
+    c->n_resblocks = 3;
+    c->rb_kernels[0] = 3;
+    c->rb_kernels[1] = 7;
+    c->rb_kernels[2] = 11;
+    c->n_dilations = 3;
+    for (int j = 0; j < 3; ++j) {
+        c->rb_dilations[j][0] = 1;
+        c->rb_dilations[j][1] = 3;
+        c->rb_dilations[j][2] = 5;
+    }
+    c->sampling_rate = 32000;
+    c->precision = MH3A_BF16X3;
+    c->flags = 0;
+    c->max_batch = 2;
+    c->max_frames = 400;
+}
+
+const char* mh3a_status_string(mh3a_status s) {
+    switch (s) {
+        case MH3A_OK: return "ok";
+        case MH3A_ERR_INVALID_ARG: return "invalid argument";
+        case MH3A_ERR_CONFIG: return "unsupported configuration";
+        case MH3A_ERR_SHAPE: return "shape mismatch";
+        case MH3A_ERR_MISSING_WEIGHT: return "missing weight";
+        case MH3A_ERR_ALLOC: return "allocation failed";
+        case MH3A_ERR_CUDA: return "CUDA error";
+        case MH3A_ERR_UNSUPPORTED: return "unsupported request";
+    }
+    return "unknown status";
+}
+
+const char* mh3a_last_error(void) { return g_last_error.c_str(); }
+
+void mh3a_destroy(mh3a_handle* h) {
+    if (!h) return;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    for (auto& e : h->ev)
+        if (e) cudaEventDestroy(e);
+    if (h->warena) cudaFree(h->warena);
+    if (h->arena) cudaFree(h->arena);
+    cudaSetDevice(prev);
+    delete h;
+}
+
+mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int n_weights, mh3a_handle** out) {
+    if (out) *out = nullptr;
+    if (!cfg || !weights || !out || n_weights < 1) return MH3A_ERR_INVALID_ARG;
+    mh3a_status st = validate(*cfg);
+    if (st) return st;
+    mh3a_handle* h = new (std::nothrow) mh3a_handle();
+    if (!h) return MH3A_ERR_ALLOC;
+    h->cfg = *cfg;
+    h->cfg.latents_mean = nullptr;  // folded below; the caller's arrays are not retained
+    h->cfg.latents_std = nullptr;
+    cudaGetDevice(&h->device);
+    build_filter(&h->filt);
+    const mh3a_config& c = h->cfg;
+    for (int i = 0; i < c.n_stages; ++i) h->hop *= c.rates[i];
+
+    Lookup lk{weights, n_weights};
+    HostArena ha;
+    auto fail = [&](mh3a_status s) {
+        mh3a_destroy(h);
+        return s;
+    };
+    // dec_in_proj with the optional denormalisation z = x * std + mean folded in:
+    //   W'[o, c] = W[o, c] std_c,   b'[o] = b[o] + sum_c W[o, c] mean_c
+    {
+        const mh3a_tensor* w = lk.find("dec_in_proj.weight");
+        const mh3a_tensor* b = lk.find("dec_in_proj.bias");
+        if (!w || !b) return fail(MH3A_ERR_MISSING_WEIGHT);
+        const int O = c.latent_dim, I = c.latent_channels;
+        if (numel(w) != (long long)O * I || numel(b) != O) return fail(MH3A_ERR_SHAPE);
+        std::vector<float> wt((size_t)I * O), bt(O);
+        for (int o = 0; o < O; ++o) {
+            double bo = b->host_data[o];
+            for (int ci = 0; ci < I; ++ci) {
+                const double wv = w->host_data[(size_t)o * I + ci];
+                const double sd = cfg->latents_std ? cfg->latents_std[ci] : 1.0;
+                const double mu = cfg->latents_mean ? cfg->latents_mean[ci] : 0.0;
+                wt[(size_t)ci * O + o] = (float)(wv * sd);
+                bo += wv * mu;
+            }
+            bt[o] = (float)bo;
+        }
+        ha.add(wt, &h->in_proj.w);
+        ha.add(bt, &h->in_proj.b);
+        h->in_proj.cin = I;
+        h->in_proj.cout = O;
+        h->in_proj.k = 1;
+    }
+    {
+        const mh3a_tensor* v = lk.find("decoder.conv_pre.weight_v");
+        if (!v) return fail(MH3A_ERR_MISSING_WEIGHT);
+        if (v->ndim != 3 || v->shape[2] != 7) return fail(MH3A_ERR_SHAPE);
+        std::vector<float> oik;
+        if ((st = fold_conv(lk, "decoder.conv_pre", c.decoder_dim, c.latent_dim, 7, true, ha, &h->pre,
+                            c.precision == MH3A_BF16X3 ? &oik : nullptr)))
+            return fail(st);
+        if (c.precision == MH3A_BF16X3) prepare_tc_pre(oik, c.decoder_dim, c.latent_dim, 7, &h->tc[0]);
+    }
+    int C = c.decoder_dim;
+    char buf[160];
+    for (int i = 0; i < c.n_stages; ++i) {
+        const int Co = C / 2;
+        std::snprintf(buf, sizeof buf, "decoder.ups.%d.0", i);
+        if ((st = fold_convT(lk, buf, C, Co, c.kernels[i], ha, &h->ups[i]))) return fail(st);
+        h->stage_tc[i] = (c.precision == MH3A_BF16X3) && tc_stage_supported(Co, c);
+        for (int j = 0; j < c.n_resblocks; ++j) {
+            const int k = c.rb_kernels[j];
+            const int rb = i * c.n_resblocks + j;
+            for (int m = 0; m < c.n_dilations; ++m) {
+                std::vector<float> oik1, oik2;
+                const bool tc = h->stage_tc[i];
+                std::snprintf(buf, sizeof buf, "decoder.resblocks.%d.convs1.%d", rb, m);
+                if ((st = fold_conv(lk, buf, Co, Co, k, true, ha, &h->rb1[i][j][m], tc ? &oik1 : nullptr)))
+                    return fail(st);
+                std::snprintf(buf, sizeof buf, "decoder.resblocks.%d.convs2.%d", rb, m);
+                if ((st = fold_conv(lk, buf, Co, Co, k, true, ha, &h->rb2[i][j][m], tc ? &oik2 : nullptr)))
+                    return fail(st);
+                if (tc) {
+                    prepare_tc_conv(oik1, Co, k, &h->tc[i].conv[j][m][0]);
+                    prepare_tc_conv(oik2, Co, k, &h->tc[i].conv[j][m][1]);
+                }
+                std::snprintf(buf, sizeof buf, "decoder.resblocks.%d.activations.%d.act", rb, 2 * m);
+                if ((st = load_act(lk, buf, Co, ha, &h->act1[i][j][m]))) return fail(st);
+                std::snprintf(buf, sizeof buf, "decoder.resblocks.%d.activations.%d.act", rb, 2 * m + 1);
+                if ((st = load_act(lk, buf, Co, ha, &h->act2[i][j][m]))) return fail(st);
+            }
+        }
+        C = Co;
+    }
+    if ((st = load_act(lk, "decoder.activation_post.act", C, ha, &h->act_post))) return fail(st);
+    {
+        const mh3a_tensor* v = lk.find("decoder.conv_post.weight_v");
+        if (!v) return fail(MH3A_ERR_MISSING_WEIGHT);
+        if (v->ndim != 3 || v->shape[2] != 7) return fail(MH3A_ERR_SHAPE);
+        if ((st = fold_conv(lk, "decoder.conv_post", 1, C, 7, false, ha, &h->post))) return fail(st);
+    }
+    // tensor-core operand copies go into the same arena
+    for (int i = 0; i < c.n_stages; ++i) tc_register(&h->tc[i], [&](const std::vector<float>& v, float** d) { ha.add(v, d); });
+
+    // one device copy of every folded weight
+    h->wbytes = ha.data.size() * sizeof(float);
+    if (cudaMalloc(&h->warena, h->wbytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
+    if (cudaMemcpy(h->warena, ha.data.data(), h->wbytes, cudaMemcpyHostToDevice) != cudaSuccess)
+        return fail(cuda_fail(cudaGetLastError(), "weight upload"));
+    for (auto& f : ha.fix) *f.dst = reinterpret_cast<float*>(h->warena) + f.off;
+    for (int i = 0; i < c.n_stages; ++i) tc_finalize(&h->tc[i]);
+
+    // workspace: stage buffers sized for the widest stage at max_batch x max_frames
+    long long cap = 0, len = 1;
+    for (int i = 0; i < c.n_stages; ++i) {
+        len *= c.rates[i];
+        const long long v = (long long)stage_channels(c, i) * len;
+        cap = cap > v ? cap : v;
+    }
+    const long long BN = (long long)c.max_batch * c.max_frames;
+    h->stage_cap = ((cap * BN + 63) / 64) * 64;
+    auto rnd = [](long long n) { return ((n + 63) / 64) * 64; };
+    const long long n_in = rnd((long long)c.latent_dim * BN), n_pre = rnd((long long)c.decoder_dim * BN);
+    const long long n_lat = rnd((long long)c.latent_channels * BN), n_wav = rnd((long long)h->hop * BN);
+    const long long nbuf = 1 + 2 * c.n_resblocks;
+    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav;
+    h->abytes = (size_t)total * sizeof(float);
+    if (cudaMalloc(&h->arena, h->abytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
+    float* p = reinterpret_cast<float*>(h->arena);
+    h->buf_in = p; p += n_in;
+    h->buf_pre = p; p += n_pre;
+    h->H = p; p += h->stage_cap;
+    for (int j = 0; j < c.n_resblocks; ++j) { h->X[j] = p; p += h->stage_cap; }
+    for (int j = 0; j < c.n_resblocks; ++j) { h->T[j] = p; p += h->stage_cap; }
+    h->lat_io = p; p += n_lat;
+    h->wav_io = p; p += n_wav;
+    for (auto& e : h->ev)
+        if (cudaEventCreate(&e) != cudaSuccess) return fail(cuda_fail(cudaGetLastError(), "cudaEventCreate"));
+    if (cudaDeviceSynchronize() != cudaSuccess) return fail(cuda_fail(cudaGetLastError(), "create"));
+    *out = h;
+    return MH3A_OK;
+}
+
+mh3a_status mh3a_decode(mh3a_handle* h, const float* latents, int B, int N, float* out, void* stream) {
+    if (!h || !latents || !out) return MH3A_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || B > h->cfg.max_batch || N > h->cfg.max_frames) return MH3A_ERR_SHAPE;
+    return run_decode(h, latents, B, N, out, (cudaStream_t)stream);
+}
+
+mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, int N, float* out_host,
+                             void* stream) {
+    if (!h || !latents_host || !out_host) return MH3A_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || B > h->cfg.max_batch || N > h->cfg.max_frames) return MH3A_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t in_bytes = (size_t)B * h->cfg.latent_channels * N * sizeof(float);
+    const size_t out_bytes = (size_t)B * h->hop * N * sizeof(float);
+    CK_CUDA(cudaMemcpyAsync(h->lat_io, latents_host, in_bytes, cudaMemcpyHostToDevice, s), "latents upload");
+    mh3a_status st = run_decode(h, h->lat_io, B, N, h->wav_io, s);
+    if (st) return st;
+    CK_CUDA(cudaMemcpyAsync(out_host, h->wav_io, out_bytes, cudaMemcpyDeviceToHost, s), "waveform download");
+    CK_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    return MH3A_OK;
+}
+
+mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L, int stage, float* out, void* stream) {
+    if (!h || !x || !out) return MH3A_ERR_INVALID_ARG;
+    if (stage < 0 || stage >= h->cfg.n_stages) return MH3A_ERR_INVALID_ARG;
+    if (B < 1 || L < 1) return MH3A_ERR_SHAPE;
+    const int C = stage_channels(h->cfg, stage);
+    if ((long long)B * C * L > h->stage_cap) return MH3A_ERR_SHAPE;
+    if (h->cfg.n_resblocks != 3) return MH3A_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    mh3a_status st = run_amp(h, stage, x, B, L, s);
+    if (st) return st;
+    Mean3Params mp{h->X[0], h->X[1], h->X[2], out, (long long)B * C * L, 0};
+    mp.vec4 = ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(h->X[0]) |
+                reinterpret_cast<uintptr_t>(h->X[1]) | reinterpret_cast<uintptr_t>(h->X[2])) & 15) == 0;
+    return counted(h, launch_mean3(mp, s));
+}
+
+mh3a_status mh3a_set_profiling(mh3a_handle* h, int enable) {
+    if (!h) return MH3A_ERR_INVALID_ARG;
+    h->profiling = enable != 0;
+    return MH3A_OK;
+}
+
+mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int* count) {
+    if (!h || !ms || !count || cap < 0) return MH3A_ERR_INVALID_ARG;
+    *count = 0;
+    if (h->nseg < 2) return MH3A_OK;
+    CK_CUDA(cudaEventSynchronize(h->ev[h->nseg - 1]), "cudaEventSynchronize");
+    const int n = h->nseg - 1;
+    for (int i = 0; i < n && i < cap; ++i) {
+        float t = 0.f;
+        CK_CUDA(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]), "cudaEventElapsedTime");
+        ms[i] = t;
+    }
+    *count = n < cap ? n : cap;
+    return MH3A_OK;
+}
+
+long long mh3a_launch_count(const mh3a_handle* h) { return h ? h->launches : -1; }
+
+long long mh3a_device_bytes(const mh3a_handle* h) { return h ? (long long)(h->wbytes + h->abytes) : -1; }
+
+}  // extern "C"

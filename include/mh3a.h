@@ -1,0 +1,171 @@
+/*
+ * mh3a.h -- C ABI of the B200 (sm_100a) BigVGAN waveform decoder of the MiniMax-H3 audio VAE.
+ *
+ * The library turns latents [B, 32, N] into a mono 32 kHz waveform [B, 1, 800 N] clamped to
+ * [-1, 1] (diffusers "AutoencoderKLMiniMaxH3Audio" page, `decode` section).  Stereo is carried
+ * as two batch items that decode independently (same page, introduction).  The network is the
+ * one the FastVideo "minimax_h3_audio_vae" page's `MLXMiniMaxH3AudioVAE.decode` evaluates:
+ * a 1x1 input projection, a weight-normed conv, seven weight-normed transposed-conv upsampling
+ * stages each followed by the average of three AMP residual blocks, a final anti-aliased
+ * SnakeBeta, a weight-normed output conv and the clamp.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are fp32, channel-first and time-contiguous: [B, C, T] row-major.
+ *   - Pointers documented as "device" must point to memory of the handle's device; pointers
+ *     documented as "host" to ordinary or pinned host memory.  The caller owns all of them;
+ *     the library never frees or retains a caller pointer past the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Device
+ *     work is enqueued on it asynchronously; the call returns before the work finishes unless
+ *     stated otherwise.
+ *   - Every entry point returns an mh3a_status.  Argument, shape and configuration errors are
+ *     detected on the host before any work is enqueued and leave outputs untouched.  Launch
+ *     failures are reported as MH3A_ERR_CUDA (the CUDA error text is available from
+ *     mh3a_last_error()).  No C++ exception crosses this boundary.
+ *   - A handle owns one workspace, so calls on one handle must not overlap in time (on
+ *     different streams or host threads).  Different handles are independent.
+ */
+#ifndef MH3A_H
+#define MH3A_H
+
+#if defined(__GNUC__)
+#define MH3A_API __attribute__((visibility("default")))
+#else
+#define MH3A_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MH3A_OK = 0,
+    MH3A_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, out-of-range index       */
+    MH3A_ERR_CONFIG = 2,         /* architecture the library cannot run (see mh3a_create) */
+    MH3A_ERR_SHAPE = 3,          /* B / N / L beyond the handle's limits, weight shapes   */
+    MH3A_ERR_MISSING_WEIGHT = 4, /* a required tensor is absent from the weight table     */
+    MH3A_ERR_ALLOC = 5,          /* device or host allocation failed                      */
+    MH3A_ERR_CUDA = 6,           /* a CUDA runtime call or kernel launch failed           */
+    MH3A_ERR_UNSUPPORTED = 7     /* valid request this build does not implement           */
+} mh3a_status;
+
+/* Arithmetic of the convolutions (activations are always computed in fp32).
+ *   MH3A_FP32     fp32 operands, fp32 accumulation, CUDA cores.
+ *   MH3A_BF16X3   tensor cores (tcgen05): each fp32 operand is split into a bf16 head and a
+ *                 bf16 tail, and the product is formed as head*head + head*tail + tail*head
+ *                 with fp32 accumulation in tensor memory (about 16 significant bits per
+ *                 operand).  Stages whose convolutions are too narrow for the tensor cores
+ *                 run the fp32 CUDA-core kernels. */
+typedef enum { MH3A_FP32 = 0, MH3A_BF16X3 = 1 } mh3a_precision;
+
+#define MH3A_FLAG_NO_CLAMP 1u /* return the waveform before the final clamp (testing)   */
+
+#define MH3A_MAX_STAGES 8
+#define MH3A_MAX_RESBLOCKS 4
+#define MH3A_MAX_DILATIONS 4
+
+/* Architecture and run-time limits.  Defaults (mh3a_default_config) are the constructor
+ * defaults of the diffusers "AutoencoderKLMiniMaxH3Audio" page. */
+typedef struct {
+    int latent_channels;                      /* 32                                       */
+    int latent_dim;                           /* 2048                                     */
+    int decoder_dim;                          /* 1024, halved by every upsampling stage   */
+    int n_stages;                             /* 7                                        */
+    int rates[MH3A_MAX_STAGES];               /* (5,5,2,2,2,2,2); product = hop = 800     */
+    int kernels[MH3A_MAX_STAGES];             /* (9,9,4,4,4,4,4)                          */
+    int n_resblocks;                          /* 3                                        */
+    int rb_kernels[MH3A_MAX_RESBLOCKS];       /* (3,7,11)                                 */
+    int n_dilations;                          /* 3                                        */
+    int rb_dilations[MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS]; /* ((1,3,5) x 3)            */
+    int sampling_rate;                        /* 32000 (informational)                    */
+    int precision;                            /* mh3a_precision                           */
+    unsigned flags;                           /* MH3A_FLAG_*                              */
+    /* Per-channel latent statistics (host, [latent_channels]) or NULL.  When given, decode
+     * first denormalises z = x * std_c + mean_c (diffusers "AutoencoderKLMiniMaxH3" page,
+     * latent normalisation bullet); the library folds this into the input projection. */
+    const float* latents_mean;
+    const float* latents_std;
+    int max_batch;                            /* workspace sizing: largest B              */
+    int max_frames;                           /* workspace sizing: largest N (latents)    */
+} mh3a_config;
+
+/* One named host tensor of the weight table.  Names are the checkpoint keys the MLX page's
+ * decode reads: "dec_in_proj.weight|bias", "decoder.conv_pre.weight_v|weight_g|bias",
+ * "decoder.ups.{i}.0.weight_v|weight_g|bias", "decoder.resblocks.{n}.convs1.{m}.weight_v|
+ * weight_g|bias", "decoder.resblocks.{n}.convs2.{m}.…", "decoder.resblocks.{n}.activations.
+ * {a}.act.alpha|beta" (a = 2m before convs1.m, 2m+1 before convs2.m),
+ * "decoder.activation_post.act.alpha|beta", "decoder.conv_post.weight_v|weight_g[|bias]".
+ * Transposed-conv weights are stored [in, out, k]; all other conv weights [out, in, k];
+ * weight_g is [dim0, 1, 1] and normalises over every axis but the first. */
+typedef struct {
+    const char* name;
+    const float* host_data;
+    int ndim;
+    long long shape[3];
+} mh3a_tensor;
+
+typedef struct mh3a_handle mh3a_handle;
+
+/* Fill *cfg with the default architecture, precision MH3A_BF16X3, no flags, no latent
+ * statistics, max_batch 2, max_frames 400. */
+MH3A_API void mh3a_default_config(mh3a_config* cfg);
+
+/* Build a decoder on the current CUDA device.  Copies the weight table to device memory,
+ * folds every weight norm w = g * v / ||v|| (MLX page `_wn_weight`) and the optional latent
+ * denormalisation into the weights, builds the Kaiser-sinc activation filter (MLX page
+ * `kaiser_sinc_filter1d`, cutoff 0.25, half-width 0.3, 12 taps) and allocates the workspace for
+ * max_batch x max_frames.  Blocks until the copies are done.  The host tensors may be freed
+ * after the call.
+ * Errors: MH3A_ERR_INVALID_ARG (NULL cfg/weights/out), MH3A_ERR_CONFIG (the product of the
+ * rates is not 800, the hop of the encoder the decoder inverts; some K_i - r_i is odd or
+ * negative, so a stage would not output exactly r_i samples per input; decoder_dim is not
+ * divisible by 2^n_stages; more stages/blocks/dilations than the MAX_* limits; an even
+ * residual-block kernel; unknown precision; non-positive max_batch or max_frames), MH3A_ERR_MISSING_WEIGHT, MH3A_ERR_SHAPE (a tensor's shape disagrees with the
+ * architecture), MH3A_ERR_ALLOC, MH3A_ERR_CUDA.  On error *out is set to NULL. */
+MH3A_API mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int n_weights,
+                        mh3a_handle** out);
+
+/* Decode latents (device, [B, latent_channels, N]) into a waveform (device, [B, 1, hop*N]),
+ * clamped to [-1, 1] unless MH3A_FLAG_NO_CLAMP was configured.  `out` must not overlap
+ * `latents`.  1 <= B <= max_batch, 1 <= N <= max_frames, else MH3A_ERR_SHAPE. */
+MH3A_API mh3a_status mh3a_decode(mh3a_handle* h, const float* latents, int B, int N, float* out,
+                        void* stream);
+
+/* The same decode from and to HOST memory: copies the latents in, decodes, copies the
+ * waveform out, all on `stream`, and waits for the stream before returning.  Pinned host
+ * buffers give the fastest copies.  Same shape limits as mh3a_decode. */
+MH3A_API mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, int N,
+                             float* out_host, void* stream);
+
+/* One AMP stage (MLX page `decode`, the averaged `_amp_block` outputs of upsampling stage
+ * `stage`): x (device, [B, C, L]) -> out (device, [B, C, L]) with C = decoder_dim /
+ * 2^(stage+1).  `out` must not overlap `x`.  B * L must not exceed the workspace, i.e.
+ * B * L <= max_batch * max_frames * (product of rates[0..stage]); else MH3A_ERR_SHAPE. */
+MH3A_API mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L, int stage, float* out,
+                           void* stream);
+
+/* Per-segment device timing.  When enabled, each decode records CUDA events between its
+ * segments (input projection, conv_pre, then per stage: upsampling, AMP stage; then the output
+ * activation+conv); mh3a_segment_times waits for the last decode and writes up to `cap`
+ * durations in milliseconds, returning the number of segments through *count. */
+MH3A_API mh3a_status mh3a_set_profiling(mh3a_handle* h, int enable);
+MH3A_API mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int* count);
+
+/* Number of kernels this handle has launched since creation (all entry points). */
+MH3A_API long long mh3a_launch_count(const mh3a_handle* h);
+
+/* Bytes of device memory the handle owns (weights + workspace). */
+MH3A_API long long mh3a_device_bytes(const mh3a_handle* h);
+
+/* Release the handle's device memory.  NULL is ignored.  Waits for the handle's work. */
+MH3A_API void mh3a_destroy(mh3a_handle* h);
+
+/* Static description of a status code. */
+MH3A_API const char* mh3a_status_string(mh3a_status s);
+
+/* Text of the last CUDA error seen by the calling host thread ("" if none). */
+MH3A_API const char* mh3a_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MH3A_H */

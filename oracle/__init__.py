@@ -73,6 +73,8 @@ def lib():
         L.orc_upsample2.argtypes = [_D, C.c_int, _D, C.c_int, _D]
         L.orc_downsample2.argtypes = [_D, C.c_int, _D, C.c_int, _D]
         L.orc_activation1d.argtypes = [_D, C.c_int, C.c_double, C.c_double, _D, C.c_int, _D]
+        L.orc_num_threads.argtypes = []
+        L.orc_num_threads.restype = C.c_int
         L.orc_default_config.argtypes = [C.POINTER(_Config)]
         L.orc_decode.argtypes = [C.POINTER(_Config), C.POINTER(_Tensor), C.c_int, _F, C.c_int,
                                  C.c_int, _D]
@@ -306,5 +308,6 @@ def amp_stage(arch, weights: dict, stage: int, x: np.ndarray) -> np.ndarray:
     return out
 
 
-def default_threads() -> int:
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(lib().orc_num_threads())

@@ -2,7 +2,7 @@
 
     python oracle/build.py            # writes oracle/libmh3a_oracle.so
 
-Plain gcc, -O2, OpenMP.  The oracle is the checker: it is compiled here but never linked
+Plain gcc, -O3, OpenMP.  The oracle is the checker: it is compiled here but never linked
 into, imported by or called from the CUDA library.
 """
 from __future__ import annotations
@@ -27,7 +27,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     # x86-64-v3 (AVX2/FMA) keeps the library portable across the hosts it is copied to;
     # -ffp-contract=off keeps each multiply and add a separately rounded fp64 operation.
     cmd = [
-        "gcc", "-O2", "-march=x86-64-v3", "-ffp-contract=off", "-fopenmp", "-fPIC",
+        "gcc", "-O3", "-march=x86-64-v3", "-ffp-contract=off", "-fopenmp", "-fPIC",
         "-shared", "-std=c11", "-Wall", "-o", tmp, SRC, "-lm",
     ]
     if verbose:

@@ -24,6 +24,7 @@
 #include "mh3a_oracle.h"
 
 #include <math.h>
+#include <omp.h>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -110,9 +111,15 @@ void orc_conv1d(const double* x, int Cin, int Lin, const double* w, int Cout, in
                 for (int j = 0; j < K; ++j) {
                     const double wv = w[((long long)o * Cin + c) * K + j];
                     const int off = j * dil - pad;
-                    for (int t = t0; t < t1; ++t) {
-                        const int s = t * stride + off;
-                        if (s >= 0 && s < Lin) yo[t] += wv * xc[s];
+                    /* the t for which the tap lands inside [0, Lin); outside it reads zero */
+                    int lo = t0, hi = t1;
+                    while (lo < hi && lo * stride + off < 0) ++lo;
+                    while (hi > lo && (hi - 1) * stride + off >= Lin) --hi;
+                    if (stride == 1) {
+                        const double* xs = xc + off;
+                        for (int t = lo; t < hi; ++t) yo[t] += wv * xs[t];
+                    } else {
+                        for (int t = lo; t < hi; ++t) yo[t] += wv * xc[t * stride + off];
                     }
                 }
             }
@@ -199,6 +206,8 @@ static void act_channels(const double* x, int C, int L, const float* alpha, cons
 /* ------------------------------------------------------------------------------------------ */
 /* Weight table lookup and the decode ([P3] `MLXMiniMaxH3AudioVAE.decode`).                     */
 /* ------------------------------------------------------------------------------------------ */
+
+int orc_num_threads(void) { return omp_get_max_threads(); }
 
 void orc_default_config(orc_config* cfg) {
     static const int rates[7] = {5, 5, 2, 2, 2, 2, 2};

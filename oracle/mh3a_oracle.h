@@ -86,6 +86,9 @@ void orc_downsample2(const double* s, int L2, const double* taps, int K, double*
 void orc_activation1d(const double* x, int L, double alpha, double beta, const double* taps,
                       int K, double* y);
 
+/* Number of OpenMP threads the oracle's parallel loops use. */
+int orc_num_threads(void);
+
 /* Default architecture ([P1] constructor defaults) with clamp on and no denormalisation. */
 void orc_default_config(orc_config* cfg);
 
