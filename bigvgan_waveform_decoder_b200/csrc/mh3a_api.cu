@@ -402,6 +402,65 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
 
 }  // namespace
 
+namespace mh3a {
+
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+int handle_device(const mh3a_handle* h) { return h->device; }
+
+int handle_stage_channels(const mh3a_handle* h, int stage) { return stage_channels(h->cfg, stage); }
+
+bool handle_stage_valid(const mh3a_handle* h, int stage) { return stage >= 0 && stage < h->cfg.n_stages; }
+
+int handle_n_resblocks(const mh3a_handle* h) { return h->cfg.n_resblocks; }
+
+// One AMP stage with caller-provided block buffers X[j] (running sums) and T[j]
+// (intermediates), each of at least B * C * L floats, then the mean of the blocks into `out`.
+mh3a_status amp_stage_into(mh3a_handle* h, const float* x, int B, int L, int stage, float* out,
+                           float* const* X, float* const* T, cudaStream_t s) {
+    const mh3a_config& c = h->cfg;
+    const int C = stage_channels(c, stage);
+    const int nrb = c.n_resblocks;
+    for (int m = 0; m < c.n_dilations; ++m) {
+        for (int half = 0; half < 2; ++half) {
+            ConvParams p{};
+            p.Cin = C;
+            p.Cout = C;
+            p.L = L;
+            p.B = B;
+            p.clamp = 0;
+            p.filt = h->filt;
+            for (int j = 0; j < nrb; ++j) {
+                const int k = c.rb_kernels[j];
+                const int d = (half == 0) ? c.rb_dilations[j][m] : 1;
+                ConvJob& J = p.job[j];
+                const DevConv& dc = (half == 0) ? h->rb1[stage][j][m] : h->rb2[stage][j][m];
+                const DevAct& da = (half == 0) ? h->act1[stage][j][m] : h->act2[stage][j][m];
+                J.x0 = (half == 0) ? (m == 0 ? x : X[j]) : T[j];
+                J.w = dc.w;
+                J.bias = dc.b;
+                J.alpha = da.alpha;
+                J.inv_beta = da.inv_beta;
+                J.res = (half == 0) ? nullptr : (m == 0 ? x : X[j]);
+                J.out = (half == 0) ? T[j] : X[j];
+                J.K = k;
+                J.dil = d;
+                J.pad = d * (k - 1) / 2;
+            }
+            const int n = h->stage_tc[stage] ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s)
+                                             : launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
+            mh3a_status st = counted(h, n);
+            if (st) return st;
+        }
+    }
+    Mean3Params mp{X[0], X[1], X[2], out, (long long)B * C * L, 0};
+    mp.vec4 = ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(X[0]) |
+                reinterpret_cast<uintptr_t>(X[1]) | reinterpret_cast<uintptr_t>(X[2])) & 15) == 0;
+    return counted(h, launch_mean3(mp, s));
+}
+
+}  // namespace mh3a
+
 extern "C" {
 
 void mh3a_default_config(mh3a_config* c) {

@@ -143,6 +143,29 @@ MH3A_API mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host,
 MH3A_API mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L, int stage, float* out,
                            void* stream);
 
+/* Allocation-free variant of mh3a_amp_stage.  The pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory at the time they run a stage -- a
+ * real-time audio thread that must never block in the driver's allocator, or a host whose
+ * device memory belongs to another framework's fixed budget.  Such a caller creates the handle
+ * once at start-up (it may pass max_batch = max_frames = 1 to keep the handle's own workspace
+ * small) and then runs stages through this call, which allocates nothing.
+ *
+ * Arguments, results and status codes are those of mh3a_amp_stage.  The six intermediate
+ * [B, C, L] buffers of the stage live in one fixed array of MH3A_STATIC_SCRATCH_BYTES in the
+ * library's device image: the CUDA runtime places it when it loads the library's code onto a
+ * GPU, and every GPU that loads the library holds it until the process exits.  B * C * L must
+ * not exceed MH3A_STATIC_SCRATCH_MAX_ELEMS, else MH3A_ERR_SHAPE (the limit and the requested
+ * size are in mh3a_last_error()).  The current device must be the handle's device, else
+ * MH3A_ERR_INVALID_ARG.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.  All
+ * calls on one device share the array and each call leaves its contents behind: calls that
+ * overlap in time on the GPU (other streams, threads or handles) race and corrupt each other's
+ * results, so serialise them. */
+#define MH3A_STATIC_SCRATCH_BYTES (64ll << 20)
+#define MH3A_STATIC_SCRATCH_MAX_ELEMS 2796160ll /* per buffer: (64 MiB / 4 / 6) rounded to 64 */
+MH3A_API mh3a_status mh3a_amp_stage_static(mh3a_handle* h, const float* x, int B, int L, int stage,
+                                           float* out, void* stream);
+
 /* Per-segment device timing.  When enabled, each decode records CUDA events between its
  * segments (input projection, conv_pre, then per stage: upsampling, AMP stage; then the output
  * activation+conv); mh3a_segment_times waits for the last decode and writes up to `cap`
