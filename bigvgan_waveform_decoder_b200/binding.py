@@ -24,7 +24,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "sh
 
 EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_decode", "mh3a_decode_host",
            "mh3a_amp_stage", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
-           "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error")
+           "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error",
+           "mh3a_stage_uses_tensor_cores", "mh3a_check_device_error")
 
 
 class mh3a_config(C.Structure):
@@ -96,6 +97,10 @@ def load():
     L.mh3a_segment_times.restype = C.c_int
     L.mh3a_launch_count.argtypes = [vp]
     L.mh3a_launch_count.restype = C.c_longlong
+    L.mh3a_stage_uses_tensor_cores.argtypes = [vp, C.c_int]
+    L.mh3a_stage_uses_tensor_cores.restype = C.c_int
+    L.mh3a_check_device_error.argtypes = [vp]
+    L.mh3a_check_device_error.restype = C.c_int
     L.mh3a_device_bytes.argtypes = [vp]
     L.mh3a_device_bytes.restype = C.c_longlong
     L.mh3a_destroy.argtypes = [vp]
@@ -233,6 +238,13 @@ class Decoder:
 
     def launch_count(self) -> int:
         return int(load().mh3a_launch_count(self._h))
+
+    def stage_uses_tensor_cores(self, stage: int) -> bool:
+        return load().mh3a_stage_uses_tensor_cores(self._h, stage) == 1
+
+    def check_device_error(self):
+        """Raise if a tensor-core kernel of this handle timed out on a pipeline wait."""
+        _check(load().mh3a_check_device_error(self._h), "device pipeline")
 
     def device_bytes(self) -> int:
         return int(load().mh3a_device_bytes(self._h))

@@ -105,6 +105,7 @@ struct mh3a_handle {
     DevAct act_post;
     TcStageWeights tc[MH3A_MAX_STAGES];   // tensor-core operand copies (BF16X3)
     bool stage_tc[MH3A_MAX_STAGES] = {};
+    bool pre_tc = false;                  // conv_pre on the tensor cores
     char* warena = nullptr;
     size_t wbytes = 0;
     // workspace
@@ -118,6 +119,7 @@ struct mh3a_handle {
     float* T[MH3A_MAX_RESBLOCKS] = {};
     float* lat_io = nullptr;   // host-API staging
     float* wav_io = nullptr;
+    int* dev_err = nullptr;    // set by a tensor-core kernel whose bounded wait timed out
     // profiling
     bool profiling = false;
     cudaEvent_t ev[kMaxSegments + 1] = {};
@@ -255,8 +257,10 @@ mh3a_status record(mh3a_handle* h, cudaStream_t s) {
 
 mh3a_status counted(mh3a_handle* h, int n) {
     if (n < 0) {
-        cudaError_t e = cudaGetLastError();
-        return cuda_fail(e == cudaSuccess ? cudaErrorLaunchFailure : e, "kernel launch");
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+        g_last_error = "a launcher refused its arguments (no kernel was launched)";
+        return MH3A_ERR_UNSUPPORTED;
     }
     h->launches += n;
     return MH3A_OK;
@@ -296,7 +300,7 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
             }
             int n;
             if (h->stage_tc[stage])
-                n = launch_conv_tc(p, nrb, h->tc[stage], m, half, s);
+                n = launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err);
             else
                 n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             mh3a_status st = counted(h, n);
@@ -342,7 +346,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = h->pre.k;
         p.job[0].dil = 1;
         p.job[0].pad = 3;
-        int n = h->stage_tc[0] ? launch_conv_pre_tc(p, h->tc[0], s) : launch_conv_simt(p, 1, false, false, s);
+        int n = h->pre_tc ? launch_conv_pre_tc(p, h->tc[0], s) : launch_conv_simt(p, 1, false, false, s);
         if ((st = counted(h, n))) return st;
         if ((st = record(h, s))) return st;
     }
@@ -447,7 +451,7 @@ mh3a_status amp_stage_into(mh3a_handle* h, const float* x, int B, int L, int sta
                 J.dil = d;
                 J.pad = d * (k - 1) / 2;
             }
-            const int n = h->stage_tc[stage] ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s)
+            const int n = h->stage_tc[stage] ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err)
                                              : launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             mh3a_status st = counted(h, n);
             if (st) return st;
@@ -641,7 +645,7 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     const long long n_in = rnd((long long)c.latent_dim * BN), n_pre = rnd((long long)c.decoder_dim * BN);
     const long long n_lat = rnd((long long)c.latent_channels * BN), n_wav = rnd((long long)h->hop * BN);
     const long long nbuf = 1 + 2 * c.n_resblocks;
-    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav;
+    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64;
     h->abytes = (size_t)total * sizeof(float);
     if (cudaMalloc(&h->arena, h->abytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
     float* p = reinterpret_cast<float*>(h->arena);
@@ -652,6 +656,9 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     for (int j = 0; j < c.n_resblocks; ++j) { h->T[j] = p; p += h->stage_cap; }
     h->lat_io = p; p += n_lat;
     h->wav_io = p; p += n_wav;
+    h->dev_err = reinterpret_cast<int*>(p);
+    if (cudaMemset(h->dev_err, 0, 64 * sizeof(float)) != cudaSuccess)
+        return fail(cuda_fail(cudaGetLastError(), "cudaMemset"));
     for (auto& e : h->ev)
         if (cudaEventCreate(&e) != cudaSuccess) return fail(cuda_fail(cudaGetLastError(), "cudaEventCreate"));
     if (cudaDeviceSynchronize() != cudaSuccess) return fail(cuda_fail(cudaGetLastError(), "create"));
@@ -718,6 +725,22 @@ mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int* count) {
 }
 
 long long mh3a_launch_count(const mh3a_handle* h) { return h ? h->launches : -1; }
+
+int mh3a_stage_uses_tensor_cores(const mh3a_handle* h, int stage) {
+    if (!h || stage < 0 || stage >= h->cfg.n_stages) return -1;
+    return h->stage_tc[stage] ? 1 : 0;
+}
+
+mh3a_status mh3a_check_device_error(mh3a_handle* h) {
+    if (!h) return MH3A_ERR_INVALID_ARG;
+    int flag = 0;
+    CK_CUDA(cudaMemcpy(&flag, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost), "read device error flag");
+    if (flag == 0) return MH3A_OK;
+    CK_CUDA(cudaMemset(h->dev_err, 0, sizeof(int)), "clear device error flag");
+    g_last_error = "a tensor-core kernel gave up waiting on its pipeline (code " + std::to_string(flag) +
+                   "); its outputs are invalid";
+    return MH3A_ERR_CUDA;
+}
 
 long long mh3a_device_bytes(const mh3a_handle* h) { return h ? (long long)(h->wbytes + h->abytes) : -1; }
 

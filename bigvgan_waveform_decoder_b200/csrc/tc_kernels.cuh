@@ -40,8 +40,9 @@ void tc_finalize(TcStageWeights* w);
 
 // Launch one AMP conv layer (dilation index m, half 0 = dilated conv, 1 = k x 1 conv) for all
 // residual blocks on the tensor cores.  Returns the number of kernels launched or -1.
+// `err` is a device int the kernel sets (non-zero) if one of its bounded waits times out.
 int launch_conv_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int m, int half,
-                   cudaStream_t s);
+                   cudaStream_t s, int* err);
 int launch_conv_pre_tc(const ConvParams& p, const TcStageWeights& w, cudaStream_t s);
 
 }  // namespace mh3a

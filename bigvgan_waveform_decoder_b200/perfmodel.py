@@ -44,14 +44,16 @@ class Segment:
         return self.conv_flops + self.act_flops
 
 
-def segments(arch, B: int, N: int, tc_stages=()) -> list[Segment]:
+def segments(arch, B: int, N: int, tc_stages=(), pre_tc: bool = False) -> list[Segment]:
+    """Segments of one decode; `tc_stages` are the AMP stages whose convolutions run on the
+    tensor cores, `pre_tc` whether conv_pre does."""
     out = []
     BN = B * N
     Cz, D, C0 = arch.latent_channels, arch.latent_dim, arch.decoder_dim
     out.append(Segment("in_proj", 2.0 * Cz * D * BN, 0, 0, F32 * ((Cz + D) * BN + Cz * D + D)))
     kp = getattr(arch, "conv_pre_kernel", 7)
     out.append(Segment("conv_pre", 2.0 * D * C0 * kp * BN, 0, 0,
-                       F32 * ((D + C0) * BN + D * C0 * kp + C0), tensor=0 in tc_stages))
+                       F32 * ((D + C0) * BN + D * C0 * kp + C0), tensor=pre_tc))
     C, L = C0, N
     nrb = len(arch.rb_kernels)
     for i, (r, K) in enumerate(zip(arch.rates, arch.kernels)):

@@ -173,6 +173,17 @@ MH3A_API mh3a_status mh3a_amp_stage_static(mh3a_handle* h, const float* x, int B
 MH3A_API mh3a_status mh3a_set_profiling(mh3a_handle* h, int enable);
 MH3A_API mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int* count);
 
+/* 1 if the AMP convolutions of `stage` run on the tensor cores for this handle, 0 if on the
+ * fp32 CUDA cores, -1 for a NULL handle or an out-of-range stage. */
+MH3A_API int mh3a_stage_uses_tensor_cores(const mh3a_handle* h, int stage);
+
+/* Waits for the device, then reports whether any tensor-core kernel of this handle gave up
+ * one of its bounded pipeline waits since the last check (MH3A_ERR_CUDA, with the reason in
+ * mh3a_last_error(); the outputs of that call are invalid) and clears the flag.  Such a
+ * timeout is a defect, never an expected outcome: every wait in those kernels has an
+ * iteration limit so that a defect ends the kernel instead of hanging the GPU. */
+MH3A_API mh3a_status mh3a_check_device_error(mh3a_handle* h);
+
 /* Number of kernels this handle has launched since creation (all entry points). */
 MH3A_API long long mh3a_launch_count(const mh3a_handle* h);
 

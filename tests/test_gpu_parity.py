@@ -87,6 +87,9 @@ def test_amp_stage_matches_oracle(dev, full_weights, stage, B, L, precision):
     d = decoder(arch, full_weights, precision, max_batch=2, max_frames=64)
     y = d.amp_stage(torch.from_numpy(x).to(dev), stage)
     torch.cuda.synchronize()
+    d.check_device_error()
+    if precision == Bd.MH3A_BF16X3:
+        assert d.stage_uses_tensor_cores(stage) == (C >= 32)
     check(y.cpu().numpy(), ref, precision, f"stage {stage}")
 
 
@@ -101,6 +104,8 @@ def test_decode_small_matches_oracle(dev, full_weights, precision):
     check(y, ref, precision, "decode N=4")
     dc = decoder(arch, w, precision, max_batch=2, max_frames=64, no_clamp=False)
     yc = dc.decode(zt).cpu().numpy()
+    d.check_device_error()
+    dc.check_device_error()
     np.testing.assert_array_equal(yc, np.clip(y, -1.0, 1.0))
     assert yc.shape == (1, 1, 3200) and np.all(np.abs(yc) <= 1.0)
 
