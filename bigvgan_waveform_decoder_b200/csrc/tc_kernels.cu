@@ -36,7 +36,7 @@ namespace {
 
 constexpr int KC = 32;              // input channels per chunk (4 groups of 8)
 constexpr int KG = KC / 8;          // channel groups per chunk
-constexpr int NPROD = 256;          // producer / epilogue threads (warps 2..9)
+constexpr int NPROD = 512;          // producer / epilogue threads (warps 2..17)
 constexpr int NTHREADS = NPROD + 64;
 constexpr int NSA = 2;              // activation pipeline depth
 constexpr int NSB = 3;              // weight pipeline depth
@@ -70,25 +70,17 @@ struct TcPlan {
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
-// sin^2(alpha u) with an exact phase, Cody-Waite reduction modulo pi and a Taylor sine
-// (the same construction as the fp32 CUDA-core kernels).
-__device__ __forceinline__ float sin_sq(float alpha, float u) {
+// sin^2(alpha u) for the tensor-core path: Cody-Waite reduction modulo pi, then the hardware
+// sine on [-pi/2, pi/2] (absolute error near 2^-21, far below the 3xBF16 operand error).
+__device__ __forceinline__ float sin_sq_fast(float alpha, float u) {
     const float kInvPi = 0.318309886183790671538f;
     const float kPiHi = 3.14159274101257324219f;
     const float kPiLo = -8.74227800037248297e-08f;
     const float v = alpha * u;
-    const float e = fmaf(alpha, u, -v);
     const float k = rintf(v * kInvPi);
     float r = fmaf(-k, kPiHi, v);
-    r = fmaf(-k, kPiLo, r) + e;
-    const float r2 = r * r;
-    float p = 1.0f / 6227020800.0f;
-    p = fmaf(p, r2, -1.0f / 39916800.0f);
-    p = fmaf(p, r2, 1.0f / 362880.0f);
-    p = fmaf(p, r2, -1.0f / 5040.0f);
-    p = fmaf(p, r2, 1.0f / 120.0f);
-    p = fmaf(p, r2, -1.0f / 6.0f);
-    const float s = fmaf(r * r2, p, r);
+    r = fmaf(-k, kPiLo, r);
+    const float s = __sinf(r);
     return s * s;
 }
 
@@ -128,8 +120,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
 
     uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
     uint8_t* Bs = smem + pl.offB;              // [NSB][2][KG][NT][16 B]
-    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [8][XWs]
-    float* sw = xs + 8 * pl.XWs;                            // [8][SWs]
+    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [2][8][XWs] (double buffer)
+    float* sw = xs + 2 * 8 * pl.XWs;                        // [8][SWs]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
     uint64_t* a_full = bars;
     uint64_t* a_empty = bars + NSA;
@@ -244,39 +236,53 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- activation producers
+        // Work is done one group of 8 input channels at a time.  Warp pair (2c, 2c+1) owns
+        // channel c of the group; its 64 lanes stride over positions.  The next group's input
+        // window is prefetched with cp.async into the other half of a double buffer while the
+        // current group is being processed.
         const int ptid = threadIdx.x - 64;
+        const int pw = ptid >> 5;                  // producer warp 0..15
+        const int ch = pw >> 1;                    // channel within the group
+        const int lane64 = ((pw & 1) << 5) | lane; // position stride index 0..63
         const int a_start = t0 - pad;
         const int xs_start = a_start - 6;
         const int n_start = 2 * a_start - 5;
         const int XW = ROWS + 12, SW = 2 * ROWS + 10;
         const long long xbase = (long long)b * C * L;
-        for (int chunk = 0; chunk < nchunks; ++chunk) {
+        const int gtotal = nchunks * KG;
+        // x window of group gi (channels gi*8 .. gi*8+7), replicate-clamped at the sequence ends
+        auto prefetch = [&](int gi) {
+            float* dst = xs + (size_t)(gi & 1) * 8 * pl.XWs + ch * pl.XWs;
+            const float* src = J.x + xbase + (long long)(gi * 8 + ch) * L;
+            for (int q = lane64; q < XW; q += 64) ptx::cp_async4(dst + q, src + clampi(xs_start + q, 0, L - 1));
+            ptx::cp_async_commit();
+        };
+        prefetch(0);
+        for (int gi = 0; gi < gtotal; ++gi) {
+            const int chunk = gi / KG, g = gi - chunk * KG;
             const int sa = chunk % NSA;
-            if (ptid == 0) {
-                bool go = *abort_flag == 0;
-                if (go && !ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) {
-                    go = false;
-                    *abort_flag = 1;
-                    atomicExch(p.err, 3);
+            if (g == 0) {
+                if (ptid == 0) {
+                    bool go = *abort_flag == 0;
+                    if (go && !ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) {
+                        go = false;
+                        *abort_flag = 1;
+                        atomicExch(p.err, 3);
+                    }
+                    *prod_go = go ? 1 : 0;
                 }
-                *prod_go = go ? 1 : 0;
             }
-            prod_sync();
-            if (*prod_go == 0) break;
-            uint8_t* a_hi = As + (size_t)sa * pl.SA;
-            uint8_t* a_lo = a_hi + (size_t)KG * RS * 16;
-            for (int g = 0; g < KG; ++g) {
-                const int cb = chunk * KC + g * 8;
-                for (int i = ptid; i < 8 * XW; i += NPROD) {
-                    const int c = i / XW, q = i - c * XW;
-                    xs[c * pl.XWs + q] = __ldg(J.x + xbase + (long long)(cb + c) * L + clampi(xs_start + q, 0, L - 1));
-                }
-                prod_sync();
-                for (int i = ptid; i < 8 * SW; i += NPROD) {
-                    const int c = i / SW, q = i - c * SW;
+            ptx::cp_async_wait_all();
+            prod_sync();   // x window of this group landed; the previous group's decimation is done
+            if (g == 0 && *prod_go == 0) break;
+            // ---- SnakeBeta of the 2x upsampled signal, one channel per warp pair
+            {
+                const float* xr0 = xs + (size_t)(gi & 1) * 8 * pl.XWs + ch * pl.XWs - xs_start;
+                float* srow = sw + ch * pl.SWs;
+                const float al = __ldg(J.alpha + gi * 8 + ch), ib = __ldg(J.inv_beta + gi * 8 + ch);
+                for (int q = lane64; q < SW; q += 64) {
                     const int n = clampi(n_start + q, 0, 2 * L - 1);
-                    const int m = n >> 1;
-                    const float* xr = xs + c * pl.XWs + (m - xs_start);
+                    const float* xr = xr0 + (n >> 1);
                     float u = 0.f;
                     if ((n & 1) == 0) {
 #pragma unroll
@@ -285,44 +291,71 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
 #pragma unroll
                         for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k], xr[3 - k], u);
                     }
-                    const float al = __ldg(J.alpha + cb + c), ib = __ldg(J.inv_beta + cb + c);
-                    sw[c * pl.SWs + q] = fmaf(sin_sq(al, u), ib, u);
+                    srow[q] = fmaf(sin_sq_fast(al, u), ib, u);
                 }
-                prod_sync();
-                for (int q = ptid; q < ROWS; q += NPROD) {
-                    const int gp = a_start + q;
-                    float a[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float v = 0.f;
-                        if (gp >= 0 && gp < L) {
-                            const float* sr = sw + c * pl.SWs + 2 * q;
-#pragma unroll
-                            for (int j = 0; j < kFilterTaps; ++j) v = fmaf(p.filt.down[j], sr[j], v);
-                        }
-                        a[c] = v;
-                    }
-                    uint4 hv, lv;
-                    float h[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) h[c] = bf16_round(a[c]);
-                    hv.x = pack_bf16(h[0], h[1]);
-                    hv.y = pack_bf16(h[2], h[3]);
-                    hv.z = pack_bf16(h[4], h[5]);
-                    hv.w = pack_bf16(h[6], h[7]);
-                    lv.x = pack_bf16(a[0] - h[0], a[1] - h[1]);
-                    lv.y = pack_bf16(a[2] - h[2], a[3] - h[3]);
-                    lv.z = pack_bf16(a[4] - h[4], a[5] - h[5]);
-                    lv.w = pack_bf16(a[6] - h[6], a[7] - h[7]);
-                    *reinterpret_cast<uint4*>(a_hi + ((size_t)g * RS + q) * 16) = hv;
-                    *reinterpret_cast<uint4*>(a_lo + ((size_t)g * RS + q) * 16) = lv;
-                }
-                prod_sync();
             }
-            ptx::fence_proxy_async_smem();
-            prod_sync();
-            if (ptid == 0) ptx::mbar_arrive(&a_full[sa]);
+            if (gi + 1 < gtotal) prefetch(gi + 1);
+            prod_sync();   // all 8 snake rows ready
+            // ---- decimate into the A operand: 2 rows x 4 channels per thread
+            {
+                uint8_t* a_hi = As + (size_t)sa * pl.SA + (size_t)g * RS * 16;
+                uint8_t* a_lo = a_hi + (size_t)KG * RS * 16;
+                const int npairs = (ROWS + 1) >> 1;
+                for (int it = ptid; it < 2 * npairs; it += NPROD) {
+                    const int rp = it >> 1, chh = it & 1;
+                    const int q0 = 2 * rp;
+                    float a0[4], a1[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2* sr = reinterpret_cast<const float2*>(sw + (4 * chh + c) * pl.SWs + 2 * q0);
+                        float s[14];
+#pragma unroll
+                        for (int j = 0; j < 7; ++j) {
+                            const float2 v2 = sr[j];
+                            s[2 * j] = v2.x;
+                            s[2 * j + 1] = v2.y;
+                        }
+                        float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < kFilterTaps; ++j) {
+                            v0 = fmaf(p.filt.down[j], s[j], v0);
+                            v1 = fmaf(p.filt.down[j], s[j + 2], v1);
+                        }
+                        a0[c] = v0;
+                        a1[c] = v1;
+                    }
+                    const int gp0 = a_start + q0;
+                    const bool in0 = gp0 >= 0 && gp0 < L, in1 = gp0 + 1 >= 0 && gp0 + 1 < L;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        if (q0 + r >= ROWS) break;
+                        float* a = r == 0 ? a0 : a1;
+                        const bool in = r == 0 ? in0 : in1;
+                        float h[4], l[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const float v = in ? a[c] : 0.f;
+                            h[c] = bf16_round(v);
+                            l[c] = v - h[c];
+                        }
+                        uint2 hv, lv;
+                        hv.x = pack_bf16(h[0], h[1]);
+                        hv.y = pack_bf16(h[2], h[3]);
+                        lv.x = pack_bf16(l[0], l[1]);
+                        lv.y = pack_bf16(l[2], l[3]);
+                        const size_t off = (size_t)(q0 + r) * 16 + chh * 8;
+                        *reinterpret_cast<uint2*>(a_hi + off) = hv;
+                        *reinterpret_cast<uint2*>(a_lo + off) = lv;
+                    }
+                }
+            }
+            if (g == KG - 1) {
+                ptx::fence_proxy_async_smem();
+                prod_sync();
+                if (ptid == 0) ptx::mbar_arrive(&a_full[sa]);
+            }
         }
+        ptx::cp_async_wait_all();
 
         // ---------------------------------------------------------------- epilogue
         if (ptid == 0) {
@@ -336,14 +369,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
         const bool epi_go = *prod_go != 0;   // identical in every producer thread
         ptx::tc_fence_after();
         const int q4 = warp & 3;                   // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;          // which half of the columns
-        constexpr int CPH = (NT / 2 >= 16) ? NT / 2 : 16;
+        const int part = (warp - 2) >> 2;          // which quarter of the columns (0..3)
+        constexpr int CPP = (NT / 4 >= 16) ? NT / 4 : 16;
         const long long obase = (long long)b * C * L;
-        if (epi_go && half * CPH < NT) {
+        if (epi_go && part * CPP < NT) {
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int t = t0 + mt * 128 + q4 * 32 + lane;
-                for (int cb = half * CPH; cb < half * CPH + CPH && cb < NT; cb += 16) {
+                for (int cb = part * CPP; cb < part * CPP + CPP && cb < NT; cb += 16) {
                     float v[16], w[16];
                     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
                     ptx::tmem_ld16(lane_addr + (uint32_t)(mt * NACC * NT + cb), v);
@@ -400,12 +433,12 @@ TcPlan make_plan(const TcParams& p, int njobs) {
     TcPlan pl{};
     pl.RS = 128 * MT + span;
     pl.XWs = pl.RS + 12;
-    pl.SWs = 2 * pl.RS + 10;
+    pl.SWs = 2 * pl.RS + 12;  // even (8-byte rows) with room for the last row pair's reads
     pl.SA = 2 * KG * pl.RS * 16;
     pl.SB = 2 * KG * NT * 16;
     pl.offB = NSA * pl.SA;
     pl.offX = pl.offB + NSB * pl.SB;
-    const int stage_bytes = 8 * (pl.XWs + pl.SWs) * 4;
+    const int stage_bytes = 8 * (2 * pl.XWs + pl.SWs) * 4;
     pl.offBar = (pl.offX + stage_bytes + 15) / 16 * 16;
     pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
     return pl;
