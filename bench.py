@@ -246,8 +246,9 @@ def run_ours(args):
     e2e_value = world * args.steps * audio_s / (float(t.item()) / 1e3)
 
     # per-segment roofline
-    tc_stages = tuple(i for i in range(arch.n_stages) if dec.stage_uses_tensor_cores(i))
-    segs = PM.segments(arch, B, N, tc_stages=tc_stages)
+    segs = PM.segments(arch, B, N)
+    for i, sgm in enumerate(segs):
+        sgm.tensor = dec.segment_uses_tensor_cores(i)
     dec.check_device_error()
     peaks = PM.measured_peaks()
     p_fp32 = PM.fp32_peak_tflops(peaks["sm_max_mhz"])

@@ -25,7 +25,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "sh
 EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_decode", "mh3a_decode_host",
            "mh3a_amp_stage", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
            "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error",
-           "mh3a_stage_uses_tensor_cores", "mh3a_check_device_error")
+           "mh3a_stage_uses_tensor_cores", "mh3a_segment_uses_tensor_cores",
+           "mh3a_check_device_error")
 
 
 class mh3a_config(C.Structure):
@@ -99,6 +100,8 @@ def load():
     L.mh3a_launch_count.restype = C.c_longlong
     L.mh3a_stage_uses_tensor_cores.argtypes = [vp, C.c_int]
     L.mh3a_stage_uses_tensor_cores.restype = C.c_int
+    L.mh3a_segment_uses_tensor_cores.argtypes = [vp, C.c_int]
+    L.mh3a_segment_uses_tensor_cores.restype = C.c_int
     L.mh3a_check_device_error.argtypes = [vp]
     L.mh3a_check_device_error.restype = C.c_int
     L.mh3a_device_bytes.argtypes = [vp]
@@ -241,6 +244,9 @@ class Decoder:
 
     def stage_uses_tensor_cores(self, stage: int) -> bool:
         return load().mh3a_stage_uses_tensor_cores(self._h, stage) == 1
+
+    def segment_uses_tensor_cores(self, segment: int) -> bool:
+        return load().mh3a_segment_uses_tensor_cores(self._h, segment) == 1
 
     def check_device_error(self):
         """Raise if a tensor-core kernel of this handle timed out on a pipeline wait."""

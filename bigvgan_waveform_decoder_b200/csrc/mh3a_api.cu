@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "mh3a_internal.cuh"
+#include "act_kernels.cuh"
 #include "tc_kernels.cuh"
 
 using namespace mh3a;
@@ -35,6 +36,12 @@ mh3a_status cuda_fail(cudaError_t e, const char* what) {
     } while (0)
 
 constexpr int kMaxSegments = 2 + 2 * MH3A_MAX_STAGES + 1;
+
+// Zero rows around each (item, channel group) of the tensor-core A operands: before the
+// sequence at least the largest conv padding, after it the largest tile overhang (2 x 128
+// rows) plus that padding.
+constexpr int kApadL = 32;
+constexpr int kApadR = 2 * 128 + 32;
 
 // Kaiser-windowed sinc low-pass of the activation (FastVideo "minimax_h3_audio_vae" page,
 // `kaiser_sinc_filter1d`): Kaiser's estimate A = 2.285 (K/2 - 1) pi (4 hw) + 7.95 of the stop-band
@@ -106,6 +113,7 @@ struct mh3a_handle {
     TcStageWeights tc[MH3A_MAX_STAGES];   // tensor-core operand copies (BF16X3)
     bool stage_tc[MH3A_MAX_STAGES] = {};
     bool pre_tc = false;                  // conv_pre on the tensor cores
+    bool ups_tc[MH3A_MAX_STAGES] = {};    // transposed convs on the tensor cores
     char* warena = nullptr;
     size_t wbytes = 0;
     // workspace
@@ -117,6 +125,9 @@ struct mh3a_handle {
     float* H = nullptr;
     float* X[MH3A_MAX_RESBLOCKS] = {};
     float* T[MH3A_MAX_RESBLOCKS] = {};
+    void* A_hi[MH3A_MAX_RESBLOCKS] = {};   // tensor-core A operands (activations, bf16 heads)
+    void* A_lo[MH3A_MAX_RESBLOCKS] = {};   //   and tails, with zero padding rows
+    long long a_cap = 0;                   // bf16 elements per A array
     float* lat_io = nullptr;   // host-API staging
     float* wav_io = nullptr;
     int* dev_err = nullptr;    // set by a tensor-core kernel whose bounded wait timed out
@@ -210,7 +221,7 @@ mh3a_status fold_conv(const Lookup& lk, const std::string& prefix, int O, int I,
 
 // Weight-normed transposed conv [I, O, K] (norm per input channel) -> [I, K, O].
 mh3a_status fold_convT(const Lookup& lk, const std::string& prefix, int I, int O, int K, HostArena& ha,
-                       DevConv* dc) {
+                       DevConv* dc, std::vector<float>* folded_iok = nullptr) {
     const mh3a_tensor* v = lk.find(prefix + ".weight_v");
     const mh3a_tensor* g = lk.find(prefix + ".weight_g");
     const mh3a_tensor* b = lk.find(prefix + ".bias");
@@ -219,13 +230,18 @@ mh3a_status fold_convT(const Lookup& lk, const std::string& prefix, int I, int O
         numel(b) != O)
         return MH3A_ERR_SHAPE;
     std::vector<float> w((size_t)I * K * O);
+    if (folded_iok) folded_iok->assign((size_t)I * O * K, 0.f);
     for (int c = 0; c < I; ++c) {
         const float* vc = v->host_data + (size_t)c * O * K;
         double ss = 0.0;
         for (long long q = 0; q < (long long)O * K; ++q) ss += (double)vc[q] * vc[q];
         const double sc = (double)g->host_data[c] / std::sqrt(ss);
         for (int o = 0; o < O; ++o)
-            for (int j = 0; j < K; ++j) w[((size_t)c * K + j) * O + o] = (float)(sc * vc[(size_t)o * K + j]);
+            for (int j = 0; j < K; ++j) {
+                const float val = (float)(sc * vc[(size_t)o * K + j]);
+                w[((size_t)c * K + j) * O + o] = val;
+                if (folded_iok) (*folded_iok)[((size_t)c * O + o) * K + j] = val;
+            }
     }
     ha.add(w, &dc->w);
     ha.add(std::vector<float>(b->host_data, b->host_data + O), &dc->b);
@@ -299,10 +315,33 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                 J.pad = d * (k - 1) / 2;
             }
             int n;
-            if (h->stage_tc[stage])
-                n = launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err);
-            else
+            if (h->stage_tc[stage]) {
+                // activation once per layer into the A operand, then the tensor-core GEMM
+                if ((long long)B * C * ((long long)L + kApadL + kApadR) > h->a_cap) {
+                    g_last_error = "batch too large for the tensor-core operand buffers (B > max_batch)";
+                    return MH3A_ERR_SHAPE;
+                }
+                ActParams ap{};
+                ap.C = C;
+                ap.L = L;
+                ap.B = B;
+                ap.pad_l = kApadL;
+                ap.pad_r = kApadR;
+                ap.filt = h->filt;
+                for (int j = 0; j < nrb; ++j) {
+                    ap.job[j].x = p.job[j].x0;
+                    ap.job[j].alpha = p.job[j].alpha;
+                    ap.job[j].inv_beta = p.job[j].inv_beta;
+                    ap.job[j].a_hi = h->A_hi[j];
+                    ap.job[j].a_lo = h->A_lo[j];
+                }
+                mh3a_status st = counted(h, launch_act_split(ap, nrb, s));
+                if (st) return st;
+                const long long Lpad = (long long)L + kApadL + kApadR;
+                n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err);
+            } else {
                 n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
+            }
             mh3a_status st = counted(h, n);
             if (st) return st;
         }
@@ -346,7 +385,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = h->pre.k;
         p.job[0].dil = 1;
         p.job[0].pad = 3;
-        int n = h->pre_tc ? launch_conv_pre_tc(p, h->tc[0], s) : launch_conv_simt(p, 1, false, false, s);
+        int n = h->pre_tc ? launch_conv_pre_tc(p, h->tc[0], s, h->dev_err) : launch_conv_simt(p, 1, false, false, s);
         if ((st = counted(h, n))) return st;
         if ((st = record(h, s))) return st;
     }
@@ -371,7 +410,8 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             // the fused mean reads exactly three block outputs; otherwise reduce explicitly
             return MH3A_ERR_UNSUPPORTED;
         }
-        if ((st = counted(h, launch_convT_simt(q, mean3, s)))) return st;
+        const int nl = h->ups_tc[i] ? launch_convT_tc(q, h->tc[i], s, h->dev_err) : launch_convT_simt(q, mean3, s);
+        if ((st = counted(h, nl))) return st;
         if ((st = record(h, s))) return st;
         C /= 2;
         L *= c.rates[i];
@@ -578,17 +618,23 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
         if (!v) return fail(MH3A_ERR_MISSING_WEIGHT);
         if (v->ndim != 3 || v->shape[2] != 7) return fail(MH3A_ERR_SHAPE);
         std::vector<float> oik;
+        h->pre_tc = c.precision == MH3A_BF16X3 && tc_pre_supported(c.decoder_dim, c.latent_dim, 7);
         if ((st = fold_conv(lk, "decoder.conv_pre", c.decoder_dim, c.latent_dim, 7, true, ha, &h->pre,
-                            c.precision == MH3A_BF16X3 ? &oik : nullptr)))
+                            h->pre_tc ? &oik : nullptr)))
             return fail(st);
-        if (c.precision == MH3A_BF16X3) prepare_tc_pre(oik, c.decoder_dim, c.latent_dim, 7, &h->tc[0]);
+        if (h->pre_tc) prepare_tc_pre(oik, c.decoder_dim, c.latent_dim, 7, &h->tc[0]);
     }
     int C = c.decoder_dim;
     char buf[160];
     for (int i = 0; i < c.n_stages; ++i) {
         const int Co = C / 2;
         std::snprintf(buf, sizeof buf, "decoder.ups.%d.0", i);
-        if ((st = fold_convT(lk, buf, C, Co, c.kernels[i], ha, &h->ups[i]))) return fail(st);
+        h->ups_tc[i] = c.precision == MH3A_BF16X3 && (i == 0 || c.n_resblocks == 3) &&
+                       tc_convt_supported(C, Co, c.rates[i], c.kernels[i]);
+        std::vector<float> iok;
+        if ((st = fold_convT(lk, buf, C, Co, c.kernels[i], ha, &h->ups[i], h->ups_tc[i] ? &iok : nullptr)))
+            return fail(st);
+        if (h->ups_tc[i]) prepare_tc_convt(iok, C, Co, c.kernels[i], c.rates[i], &h->tc[i].ups);
         h->stage_tc[i] = (c.precision == MH3A_BF16X3) && tc_stage_supported(Co, c);
         for (int j = 0; j < c.n_resblocks; ++j) {
             const int k = c.rb_kernels[j];
@@ -645,7 +691,13 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     const long long n_in = rnd((long long)c.latent_dim * BN), n_pre = rnd((long long)c.decoder_dim * BN);
     const long long n_lat = rnd((long long)c.latent_channels * BN), n_wav = rnd((long long)h->hop * BN);
     const long long nbuf = 1 + 2 * c.n_resblocks;
-    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64;
+    // tensor-core A operands: per block, heads and tails of B x C x (L + padding rows) bf16
+    int cmax_tc = 0;
+    for (int i = 0; i < c.n_stages; ++i)
+        if (h->stage_tc[i]) cmax_tc = std::max(cmax_tc, stage_channels(c, i));
+    h->a_cap = cmax_tc ? h->stage_cap + (long long)c.max_batch * cmax_tc * (kApadL + kApadR) : 0;
+    const long long n_a = rnd((h->a_cap + 1) / 2);   // floats per head or tail array
+    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64 + 2 * c.n_resblocks * n_a;
     h->abytes = (size_t)total * sizeof(float);
     if (cudaMalloc(&h->arena, h->abytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
     float* p = reinterpret_cast<float*>(h->arena);
@@ -656,6 +708,10 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     for (int j = 0; j < c.n_resblocks; ++j) { h->T[j] = p; p += h->stage_cap; }
     h->lat_io = p; p += n_lat;
     h->wav_io = p; p += n_wav;
+    for (int j = 0; j < c.n_resblocks && n_a > 0; ++j) {
+        h->A_hi[j] = p; p += n_a;
+        h->A_lo[j] = p; p += n_a;
+    }
     h->dev_err = reinterpret_cast<int*>(p);
     if (cudaMemset(h->dev_err, 0, 64 * sizeof(float)) != cudaSuccess)
         return fail(cuda_fail(cudaGetLastError(), "cudaMemset"));
@@ -729,6 +785,16 @@ long long mh3a_launch_count(const mh3a_handle* h) { return h ? h->launches : -1;
 int mh3a_stage_uses_tensor_cores(const mh3a_handle* h, int stage) {
     if (!h || stage < 0 || stage >= h->cfg.n_stages) return -1;
     return h->stage_tc[stage] ? 1 : 0;
+}
+
+int mh3a_segment_uses_tensor_cores(const mh3a_handle* h, int segment) {
+    if (!h) return -1;
+    const int n = 2 + 2 * h->cfg.n_stages + 1;
+    if (segment < 0 || segment >= n) return -1;
+    if (segment == 0 || segment == n - 1) return 0;   // input projection, output conv
+    if (segment == 1) return h->pre_tc ? 1 : 0;
+    const int i = (segment - 2) / 2;
+    return ((segment - 2) % 2 == 0 ? h->ups_tc[i] : h->stage_tc[i]) ? 1 : 0;
 }
 
 mh3a_status mh3a_check_device_error(mh3a_handle* h) {

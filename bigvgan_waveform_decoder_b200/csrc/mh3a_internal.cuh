@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
-#include "../../include/mh3a.h"
+#include "mh3a.h"  // include/ is on the include path
 
 namespace mh3a {
 

@@ -143,48 +143,57 @@ k_conv_simt(const ConvParams p, const SmemPlan sp) {
 #pragma unroll
             for (int i = 0; i < RT; ++i) acc[r][i] = 0.f;
         if (ACT) {
+            // The 8 warps of the block own the 8 channels of the chunk (NT == 32 * CK), so the
+            // three steps below touch only their own warp's rows and need no block barrier.
+            const int c = tid >> 5, lane = tid & 31;
+            float* xrow = xs + c * sp.XW;
+            float* srow = sw + c * sp.SW;
+            const bool live = c0 + c < Cin;
             // 1. raw input window, replicate-clamped at the sequence ends
-            for (int i = tid; i < CK * XW; i += NT) {
-                const int c = i / XW, q = i - c * XW;
-                float v = 0.f;
-                if (c0 + c < Cin) {
-                    const int g = clampi(xs_start + q, 0, L - 1);
-                    v = load_in(J.x0, J.x1, J.x2, in_base + (long long)(c0 + c) * L + g, MEAN3);
-                }
-                xs[c * sp.XW + q] = v;
-            }
-            __syncthreads();
-            // 2. SnakeBeta of the 2x upsampled signal over the decimator's window
-            for (int i = tid; i < CK * SW; i += NT) {
-                const int c = i / SW, q = i - c * SW;
-                float s = 0.f;
-                if (c0 + c < Cin) {
-                    const int n = clampi(n_start + q, 0, 2 * L - 1);
-                    const int m = n >> 1;
-                    const float* xr = xs + c * sp.XW + (m - xs_start);
-                    float u = 0.f;
-                    if ((n & 1) == 0) {
+            for (int q = lane; q < XW; q += 32)
+                xrow[q] = live ? load_in(J.x0, J.x1, J.x2,
+                                         in_base + (long long)(c0 + c) * L + clampi(xs_start + q, 0, L - 1), MEAN3)
+                               : 0.f;
+            __syncwarp();
+            // 2. SnakeBeta of the 2x upsampled signal over the decimator's window.  A lane takes
+            //    one input position m and forms both phases n = 2m, 2m+1 from x[m-3 .. m+3];
+            //    positions past either end repeat the end sample (replicate padding).
+            {
+                const float al = live ? __ldg(J.alpha + c0 + c) : 0.f;
+                const float ib = live ? __ldg(J.inv_beta + c0 + c) : 0.f;
+                const float* xr0 = xrow - xs_start;
+                const int m_lo = n_start >> 1, m_hi = (n_start + SW - 1) >> 1;
+                for (int m = m_lo + lane; m <= m_hi; m += 32) {
+                    const int mc = clampi(m, 0, L - 1);
+                    float xv[7];
 #pragma unroll
-                        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k + 1], xr[2 - k], u);
-                    } else {
+                    for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
+                    float ue = 0.f, uo = 0.f;
 #pragma unroll
-                        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k], xr[3 - k], u);
+                    for (int k = 0; k < 6; ++k) {
+                        ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
+                        uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
                     }
-                    const float al = __ldg(J.alpha + c0 + c), ib = __ldg(J.inv_beta + c0 + c);
-                    s = fmaf(sin_sq(al, u), ib, u);
+                    const float se = fmaf(sin_sq(al, ue), ib, ue);
+                    const float so = fmaf(sin_sq(al, uo), ib, uo);
+                    const int ie = 2 * m - n_start;
+                    if (ie >= 0 && ie < SW) srow[ie] = (m > L - 1) ? so : se;
+                    if (ie + 1 >= 0 && ie + 1 < SW) srow[ie + 1] = (m < 0) ? se : so;
                 }
-                sw[c * sp.SW + q] = s;
             }
-            __syncthreads();
+            __syncwarp();
             // 3. decimate into the conv window (zero outside the sequence)
-            for (int i = tid; i < CK * AW; i += NT) {
-                const int c = i / AW, q = i - c * AW;
+            for (int q = lane; q < AW; q += 32) {
                 const int g = a_start + q;
                 float a = 0.f;
                 if (g >= 0 && g < L) {
-                    const float* sr = sw + c * sp.SW + 2 * q;
+                    const float2* sr = reinterpret_cast<const float2*>(srow + 2 * q);
 #pragma unroll
-                    for (int j = 0; j < kFilterTaps; ++j) a = fmaf(p.filt.down[j], sr[j], a);
+                    for (int j = 0; j < kFilterTaps / 2; ++j) {
+                        const float2 v = sr[j];
+                        a = fmaf(p.filt.down[2 * j], v.x, a);
+                        a = fmaf(p.filt.down[2 * j + 1], v.y, a);
+                    }
                 }
                 as[c * sp.AWs + q] = a;
             }

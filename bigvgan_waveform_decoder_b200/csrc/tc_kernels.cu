@@ -1,28 +1,42 @@
-// tc_kernels.cu -- tensor-core (tcgen05 / TMEM) path of the AMP-stage convolutions.
+// tc_kernels.cu -- tensor-core (tcgen05 / TMEM) convolutions of the decode.
 //
-// One launch runs one conv layer of every residual block of an AMP stage (blockIdx.z = block,
-// heaviest kernel first).  For block j the layer is
-//   y[o, t] = bias[o] + sum_{c, tap} W[o, c, tap] * a[c, t + tap*dil - pad]  (+ residual[o, t])
-//   a = down2(snake(up2(x)))   -- the anti-aliased SnakeBeta of the FastVideo
-//                                 "minimax_h3_audio_vae" page's `_activation1d`
-// as an implicit GEMM D[t, o] = sum_k A[t, k] B[o, k] with M = time (128-row accumulators in
-// tensor memory, MT of them per CTA), N = output channels (NT per CTA), K = input channels x
-// taps.
+// One kernel template, three modes, all implicit GEMMs D[row, o] = sum_k A[row, k] B[o, k]
+// with M = time rows (128-row accumulators in tensor memory, MT of them per CTA), N = output
+// channels (NT per CTA) and K = input channels x taps:
+//
+//  AMP    one conv layer of every residual block of an AMP stage (blockIdx.z = block, the
+//         heaviest kernel first):
+//           y[o, t] = bias[o] + sum_{c, tap} W[o, c, tap] a[c, t + tap*dil - pad] (+ res[o, t])
+//         with a = down2(snake(up2(x))), the anti-aliased SnakeBeta of the FastVideo
+//         "minimax_h3_audio_vae" page's `_activation1d`, computed by the producer warps.
+//  PLAIN  the same conv without the activation (conv_pre: k = 7, padding 3).
+//  CONVT  a weight-normed transposed conv (`ups.i.0`) in polyphase form: output t = r u + phi
+//         only meets taps j = (phi + pad) mod r + r m, and reads input u + (phi + pad - j) / r.
+//         Every tap therefore is a plain shifted-window product over the input rows, so no zero
+//         is ever inserted or multiplied; each phase owns its own accumulators, and the epilogue
+//         writes phase phi of row u to output sample r u + phi.
 //
 // Precision (3xBF16): every fp32 operand is split into a bf16 head h = bf16(v) and a bf16
 // tail l = bf16(v - h); the product is accumulated as A_h B_h + A_h B_l + A_l B_h in fp32.
 //
-// Shared-memory operands use the no-swizzle K-major canonical layout: core matrices of 8 rows
-// x 16 bytes (8 bf16 along K).  The activation window is stored with ALL its rows 16 bytes
-// apart inside each 8-channel group, so the operand for tap `tap` is the same window started
-// `tap * dil` rows later: only the descriptor start address moves, and no data is copied per
-// tap.  Weights are pre-split and pre-laid-out at create time in exactly that layout, one
-// contiguous block per (output tile, 32-channel chunk, tap), so one 1-D bulk copy stages it.
+// Accumulation: the tensor core rounds its fp32 accumulator toward zero at every instruction,
+// so a long K loop into one accumulator builds a bias of about (instructions) x 2^-24
+// relative.  Each (M tile, phase) therefore owns NACC accumulators of NT columns: head x head
+// products rotate over the first NACC-1 by chunk, and the small cross terms (head x tail,
+// tail x head) go to the last one; the epilogue adds them in fp32 with round-to-nearest.
 //
-// Warp roles: warp 0 -- TMEM allocation and the MMA issuer (one thread); warp 1 -- weight
-// bulk copies (one thread); warps 2..9 -- activation producers, then the epilogue (TMEM ->
-// registers -> bias + residual -> coalesced fp32 stores along time).  Every mbarrier wait is
-// bounded; a timeout raises the error flag, and the kernel drains and returns.
+// Shared-memory operands use the no-swizzle K-major canonical layout: core matrices of 8 rows
+// x 16 bytes (8 bf16 along K).  The input window is stored with ALL its rows 16 bytes apart
+// inside each 8-channel group, so the operand of any tap is the same window started a few rows
+// later: only the descriptor start address moves.  Weights are pre-split and pre-laid-out at
+// create time in that layout, one contiguous block per (output tile, 32-channel chunk, tap),
+// so one 1-D bulk copy stages it.
+//
+// Warp roles: warp 0 -- TMEM allocation and the MMA issuer (one thread); warp 1 -- weight bulk
+// copies (one thread); warps 2..17 -- input producers (cp.async prefetch of the next 8-channel
+// window, activation or plain split into the A operand), then the epilogue (TMEM -> registers
+// -> bias + residual -> fp32 stores along time).  Every mbarrier wait is bounded; a timeout
+// raises the error flag, and the kernel drains and returns.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -42,8 +56,12 @@ constexpr int NSA = 2;              // activation pipeline depth
 constexpr int NSB = 3;              // weight pipeline depth
 constexpr uint64_t kWaitLimit = 1000000000ull;  // ns; legitimate waits last milliseconds
 
+enum Mode : int { MODE_AMP = 0, MODE_PLAIN = 1, MODE_CONVT = 2 };
+
 struct TcJob {
-    const float* x;
+    const float* x0;
+    const float* x1;     // with x2: the input is (x0 + x1 + x2) / 3 (CONVT after an AMP stage)
+    const float* x2;
     const uint16_t* w;   // pre-split operand blocks
     const float* bias;
     const float* alpha;
@@ -55,13 +73,17 @@ struct TcJob {
 
 struct TcParams {
     TcJob job[MH3A_MAX_RESBLOCKS];
-    int C, L, B, tiles_t;
+    int Cin, Cout;
+    int L;               // input length (= output length except CONVT: output r * L)
+    int B, tiles_t;
+    int r;               // CONVT rate (1 otherwise)
+    int lo;              // CONVT: window rows before the tile (the largest negative tap shift)
     ActFilter filt;
     int* err;
 };
 
 struct TcPlan {
-    int RS;         // activation rows per channel group (max over jobs)
+    int RS;         // window rows per channel group (max over jobs)
     int XWs, SWs;   // staging strides (floats)
     int SA, SB;     // bytes per activation / weight pipeline stage
     int offB, offX, offBar;
@@ -69,6 +91,8 @@ struct TcPlan {
 };
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+__device__ __forceinline__ int floordiv(int a, int r) { return (a >= 0) ? a / r : -((-a + r - 1) / r); }
 
 // sin^2(alpha u) for the tensor-core path: Cody-Waite reduction modulo pi, then the hardware
 // sine on [-pi/2, pi/2] (absolute error near 2^-21, far below the 3xBF16 operand error).
@@ -94,34 +118,48 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
 
 __device__ __forceinline__ float bf16_round(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-// Accumulation: the tensor core rounds its fp32 accumulator toward zero at every instruction,
-// so a long K loop into one accumulator builds a bias of about (instructions) x 2^-24
-// relative.  Each M tile therefore owns NACC accumulators of NT columns: head x head products
-// rotate over the first NACC-1 by chunk, and the small cross terms (head x tail, tail x head)
-// go to the last one; the epilogue adds them in fp32 with round-to-nearest.
-template <int MT, int NT, int NACC>
-__global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, const TcPlan pl) {
+// Row shift (in window rows) and phase of tap j.
+template <int MODE>
+__device__ __forceinline__ void tap_geometry(int j, int dil, int pad, int r, int lo, int& shift, int& phase,
+                                             bool& first) {
+    if (MODE == MODE_CONVT) {
+        phase = ((j - pad) % r + r) % r;
+        shift = floordiv(phase + pad - j, r) + lo;
+        first = j == (phase + pad) % r;   // the smallest tap of this phase
+    } else {
+        phase = 0;
+        shift = j * dil;
+        first = j == 0;
+    }
+}
+
+template <int MODE, int MT, int NT, int NACC, int R>
+__global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const TcPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int NHH = NACC - 1;
-    constexpr int USED = MT * NT * NACC;
+    constexpr int USED = MT * R * NT * NACC;
     static_assert(NACC >= 2 && USED <= 512, "tensor memory holds 512 columns");
     constexpr int NCOLS = (USED <= 32) ? 32 : (USED <= 64) ? 64 : (USED <= 128) ? 128 : (USED <= 256) ? 256 : 512;
+    constexpr int NIN = (MODE == MODE_CONVT) ? 3 : 1;   // staged input buffers (CONVT may average 3)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TcJob& J = p.job[blockIdx.z];
     const int K = J.K, dil = J.dil, pad = J.pad;
-    const int C = p.C, L = p.L;
+    const int Cin = p.Cin, Cout = p.Cout, L = p.L;
     const int b = blockIdx.x / p.tiles_t;
     const int t0 = (blockIdx.x % p.tiles_t) * (128 * MT);
     const int o_tile = blockIdx.y;
     const int o0 = o_tile * NT;
-    const int nchunks = C / KC;
-    const int ROWS = 128 * MT + (K - 1) * dil;
+    const int nchunks = Cin / KC;
+    const int span = (MODE == MODE_CONVT) ? (pl.RS - 128 * MT) : (K - 1) * dil;
+    const int ROWS = 128 * MT + span;
     const int RS = pl.RS;
+    const int r = (MODE == MODE_CONVT) ? p.r : 1;
+    const bool mean3 = (MODE == MODE_CONVT) && J.x1 != nullptr;
 
     uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
     uint8_t* Bs = smem + pl.offB;              // [NSB][2][KG][NT][16 B]
-    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [2][8][XWs] (double buffer)
-    float* sw = xs + 2 * 8 * pl.XWs;                        // [8][SWs]
+    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [2][NIN][8][XWs] (double buffer)
+    float* sw = xs + 2 * NIN * 8 * pl.XWs;                  // [8][SWs] (AMP only)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
     uint64_t* a_full = bars;
     uint64_t* a_empty = bars + NSA;
@@ -176,6 +214,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
                     const int sb = u % NSB;
                     if (!ptx::mbar_wait(&b_full[sb], (u / NSB) & 1, kWaitLimit)) { ok = false; break; }
                     ptx::tc_fence_after();
+                    int shift, phase;
+                    bool first;
+                    tap_geometry<MODE>(tap, dil, pad, r, p.lo, shift, phase, first);
                     const uint32_t b_hi = b_smem + sb * pl.SB;
                     const uint32_t b_lo = b_hi + KG * NT * 16;
 #pragma unroll
@@ -185,13 +226,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
                         const uint64_t bl = ptx::smem_desc(b_lo + boff, NT * 16, 128);
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
-                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + tap * dil) * 16;
+                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + shift) * 16;
                             const uint64_t ah = ptx::smem_desc(a_hi + aoff, RS * 16, 128);
                             const uint64_t al = ptx::smem_desc(a_lo + aoff, RS * 16, 128);
-                            const uint32_t dh = tmem + (uint32_t)((mt * NACC + chunk % NHH) * NT);
-                            const uint32_t dx = tmem + (uint32_t)((mt * NACC + NHH) * NT);
-                            const uint32_t acc_h = (chunk >= NHH || tap > 0 || kk > 0) ? 1u : 0u;
-                            const uint32_t acc_x = (chunk > 0 || tap > 0 || kk > 0) ? 1u : 0u;
+                            const int accbase = (mt * R + phase) * NACC;
+                            const uint32_t dh = tmem + (uint32_t)((accbase + chunk % NHH) * NT);
+                            const uint32_t dx = tmem + (uint32_t)((accbase + NHH) * NT);
+                            const uint32_t acc_h = (chunk >= NHH || !first || kk > 0) ? 1u : 0u;
+                            const uint32_t acc_x = (chunk > 0 || !first || kk > 0) ? 1u : 0u;
                             ptx::mma_bf16(dh, ah, bh, idesc, acc_h);
                             ptx::mma_bf16(dx, ah, bl, idesc, acc_x);
                             ptx::mma_bf16(dx, al, bh, idesc, 1u);
@@ -235,7 +277,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- activation producers
+        // ---------------------------------------------------------------- input producers
         // Work is done one group of 8 input channels at a time.  Warp pair (2c, 2c+1) owns
         // channel c of the group; its 64 lanes stride over positions.  The next group's input
         // window is prefetched with cp.async into the other half of a double buffer while the
@@ -244,70 +286,85 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
         const int pw = ptid >> 5;                  // producer warp 0..15
         const int ch = pw >> 1;                    // channel within the group
         const int lane64 = ((pw & 1) << 5) | lane; // position stride index 0..63
-        const int a_start = t0 - pad;
-        const int xs_start = a_start - 6;
+        const int a_start = (MODE == MODE_CONVT) ? t0 - p.lo : t0 - pad;   // first window row
+        const int xs_start = (MODE == MODE_AMP) ? a_start - 6 : a_start;   // first staged sample
         const int n_start = 2 * a_start - 5;
-        const int XW = ROWS + 12, SW = 2 * ROWS + 10;
-        const long long xbase = (long long)b * C * L;
+        const int XW = (MODE == MODE_AMP) ? ROWS + 12 : ROWS;
+        const int SW = 2 * ROWS + 10;
+        const long long xbase = (long long)b * Cin * L;
         const int gtotal = nchunks * KG;
-        // x window of group gi (channels gi*8 .. gi*8+7), replicate-clamped at the sequence ends
         auto prefetch = [&](int gi) {
-            float* dst = xs + (size_t)(gi & 1) * 8 * pl.XWs + ch * pl.XWs;
-            const float* src = J.x + xbase + (long long)(gi * 8 + ch) * L;
-            for (int q = lane64; q < XW; q += 64) ptx::cp_async4(dst + q, src + clampi(xs_start + q, 0, L - 1));
+            const long long rowoff = xbase + (long long)(gi * 8 + ch) * L;
+#pragma unroll
+            for (int s = 0; s < NIN; ++s) {
+                if (s > 0 && !mean3) break;
+                const float* src = (s == 0 ? J.x0 : (s == 1 ? J.x1 : J.x2)) + rowoff;
+                float* dst = xs + ((size_t)((gi & 1) * NIN + s) * 8 + ch) * pl.XWs;
+                for (int q = lane64; q < XW; q += 64) ptx::cp_async4(dst + q, src + clampi(xs_start + q, 0, L - 1));
+            }
             ptx::cp_async_commit();
         };
         prefetch(0);
         for (int gi = 0; gi < gtotal; ++gi) {
             const int chunk = gi / KG, g = gi - chunk * KG;
             const int sa = chunk % NSA;
-            if (g == 0) {
-                if (ptid == 0) {
-                    bool go = *abort_flag == 0;
-                    if (go && !ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) {
-                        go = false;
-                        *abort_flag = 1;
-                        atomicExch(p.err, 3);
-                    }
-                    *prod_go = go ? 1 : 0;
+            if (g == 0 && ptid == 0) {
+                bool go = *abort_flag == 0;
+                if (go && !ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) {
+                    go = false;
+                    *abort_flag = 1;
+                    atomicExch(p.err, 3);
                 }
+                *prod_go = go ? 1 : 0;
             }
             ptx::cp_async_wait_all();
-            prod_sync();   // x window of this group landed; the previous group's decimation is done
+            prod_sync();   // this group's window landed; the previous group's stores are done
             if (g == 0 && *prod_go == 0) break;
-            // ---- SnakeBeta of the 2x upsampled signal, one channel per warp pair
-            {
-                const float* xr0 = xs + (size_t)(gi & 1) * 8 * pl.XWs + ch * pl.XWs - xs_start;
-                float* srow = sw + ch * pl.SWs;
-                const float al = __ldg(J.alpha + gi * 8 + ch), ib = __ldg(J.inv_beta + gi * 8 + ch);
-                for (int q = lane64; q < SW; q += 64) {
-                    const int n = clampi(n_start + q, 0, 2 * L - 1);
-                    const float* xr = xr0 + (n >> 1);
-                    float u = 0.f;
-                    if ((n & 1) == 0) {
+            uint8_t* a_hi = As + (size_t)sa * pl.SA + (size_t)g * RS * 16;
+            uint8_t* a_lo = a_hi + (size_t)KG * RS * 16;
+            const float* xg = xs + (size_t)(gi & 1) * NIN * 8 * pl.XWs;
+            if (MODE == MODE_AMP) {
+                // ---- SnakeBeta of the 2x upsampled signal, one channel per warp pair.  A lane
+                // takes one input position m and forms both phases n = 2m (taps 1,3,..,11 on
+                // x[m+2..m-3]) and n = 2m+1 (taps 0,2,..,10 on x[m+3..m-2]) from the same seven
+                // inputs; positions past either end repeat the end sample (replicate padding).
+                {
+                    const float* xr0 = xg + ch * pl.XWs - xs_start;
+                    float* srow = sw + ch * pl.SWs;
+                    const float al = __ldg(J.alpha + gi * 8 + ch), ib = __ldg(J.inv_beta + gi * 8 + ch);
+                    const int m_lo = n_start >> 1, m_hi = (n_start + SW - 1) >> 1;
+                    for (int m = m_lo + lane64; m <= m_hi; m += 64) {
+                        const int mc = clampi(m, 0, L - 1);
+                        const float* xr = xr0 + mc;
+                        float xv[7];
 #pragma unroll
-                        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k + 1], xr[2 - k], u);
-                    } else {
+                        for (int k = 0; k < 7; ++k) xv[k] = xr[k - 3];   // x[mc-3 .. mc+3]
+                        float ue = 0.f, uo = 0.f;
 #pragma unroll
-                        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k], xr[3 - k], u);
+                        for (int k = 0; k < 6; ++k) {
+                            ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
+                            uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
+                        }
+                        const float se = fmaf(sin_sq_fast(al, ue), ib, ue);
+                        const float so = fmaf(sin_sq_fast(al, uo), ib, uo);
+                        const int ie = 2 * m - n_start;
+                        const float ve = (m > L - 1) ? so : se;
+                        const float vo = (m < 0) ? se : so;
+                        if (ie >= 0 && ie < SW) srow[ie] = ve;
+                        if (ie + 1 >= 0 && ie + 1 < SW) srow[ie + 1] = vo;
                     }
-                    srow[q] = fmaf(sin_sq_fast(al, u), ib, u);
                 }
-            }
-            if (gi + 1 < gtotal) prefetch(gi + 1);
-            prod_sync();   // all 8 snake rows ready
-            // ---- decimate into the A operand: 2 rows x 4 channels per thread
-            {
-                uint8_t* a_hi = As + (size_t)sa * pl.SA + (size_t)g * RS * 16;
-                uint8_t* a_lo = a_hi + (size_t)KG * RS * 16;
+                if (gi + 1 < gtotal) prefetch(gi + 1);
+                prod_sync();   // all 8 snake rows ready
+                // ---- decimate into the A operand: 2 rows x 2 channels per thread
                 const int npairs = (ROWS + 1) >> 1;
-                for (int it = ptid; it < 2 * npairs; it += NPROD) {
-                    const int rp = it >> 1, chh = it & 1;
+                for (int it = ptid; it < 4 * npairs; it += NPROD) {
+                    const int rp = it >> 2, cq = it & 3;   // row pair, channel pair
                     const int q0 = 2 * rp;
-                    float a0[4], a1[4];
+                    float a0[2], a1[2];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float2* sr = reinterpret_cast<const float2*>(sw + (4 * chh + c) * pl.SWs + 2 * q0);
+                    for (int c = 0; c < 2; ++c) {
+                        const float2* sr = reinterpret_cast<const float2*>(sw + (2 * cq + c) * pl.SWs + 2 * q0);
                         float s[14];
 #pragma unroll
                         for (int j = 0; j < 7; ++j) {
@@ -324,29 +381,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
                         a0[c] = v0;
                         a1[c] = v1;
                     }
-                    const int gp0 = a_start + q0;
-                    const bool in0 = gp0 >= 0 && gp0 < L, in1 = gp0 + 1 >= 0 && gp0 + 1 < L;
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        if (q0 + r >= ROWS) break;
-                        float* a = r == 0 ? a0 : a1;
-                        const bool in = r == 0 ? in0 : in1;
-                        float h[4], l[4];
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int q = q0 + rr;
+                        if (q >= ROWS) break;
+                        const bool in = a_start + q >= 0 && a_start + q < L;   // conv zero padding
+                        float h[2], l[2];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const float v = in ? a[c] : 0.f;
+                        for (int c = 0; c < 2; ++c) {
+                            const float v = in ? (rr == 0 ? a0[c] : a1[c]) : 0.f;
                             h[c] = bf16_round(v);
                             l[c] = v - h[c];
                         }
-                        uint2 hv, lv;
-                        hv.x = pack_bf16(h[0], h[1]);
-                        hv.y = pack_bf16(h[2], h[3]);
-                        lv.x = pack_bf16(l[0], l[1]);
-                        lv.y = pack_bf16(l[2], l[3]);
-                        const size_t off = (size_t)(q0 + r) * 16 + chh * 8;
-                        *reinterpret_cast<uint2*>(a_hi + off) = hv;
-                        *reinterpret_cast<uint2*>(a_lo + off) = lv;
+                        const size_t off = (size_t)q * 16 + cq * 4;
+                        *reinterpret_cast<uint32_t*>(a_hi + off) = pack_bf16(h[0], h[1]);
+                        *reinterpret_cast<uint32_t*>(a_lo + off) = pack_bf16(l[0], l[1]);
                     }
+                }
+            } else {
+                if (gi + 1 < gtotal) prefetch(gi + 1);
+                // ---- plain split of the staged input: one row (8 channels) per thread
+                for (int q = ptid; q < ROWS; q += NPROD) {
+                    const bool in = a_start + q >= 0 && a_start + q < L;   // zero outside the input
+                    float h[8], l[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float v = xg[c * pl.XWs + q];
+                        if (mean3)
+                            v = (v + xg[(8 + c) * pl.XWs + q] + xg[(16 + c) * pl.XWs + q]) / 3.0f;
+                        v = in ? v : 0.f;
+                        h[c] = bf16_round(v);
+                        l[c] = v - h[c];
+                    }
+                    uint4 hv, lv;
+                    hv.x = pack_bf16(h[0], h[1]);
+                    hv.y = pack_bf16(h[2], h[3]);
+                    hv.z = pack_bf16(h[4], h[5]);
+                    hv.w = pack_bf16(h[6], h[7]);
+                    lv.x = pack_bf16(l[0], l[1]);
+                    lv.y = pack_bf16(l[2], l[3]);
+                    lv.z = pack_bf16(l[4], l[5]);
+                    lv.w = pack_bf16(l[6], l[7]);
+                    *reinterpret_cast<uint4*>(a_hi + (size_t)q * 16) = hv;
+                    *reinterpret_cast<uint4*>(a_lo + (size_t)q * 16) = lv;
                 }
             }
             if (g == KG - 1) {
@@ -371,14 +448,239 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_amp_conv_tc(const TcParams p, c
         const int q4 = warp & 3;                   // TMEM lane quarter this warp may access
         const int part = (warp - 2) >> 2;          // which quarter of the columns (0..3)
         constexpr int CPP = (NT / 4 >= 16) ? NT / 4 : 16;
-        const long long obase = (long long)b * C * L;
+        const int Lout = L * r;
+        const long long obase = (long long)b * Cout * Lout;
         if (epi_go && part * CPP < NT) {
+            const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int row = t0 + mt * 128 + q4 * 32 + lane;
+                for (int phase = 0; phase < R; ++phase) {
+                    const int t = (MODE == MODE_CONVT) ? row * r + phase : row;
+                    for (int cb = part * CPP; cb < part * CPP + CPP && cb < NT; cb += 16) {
+                        float v[16], w[16];
+                        const int accbase = (mt * R + phase) * NACC;
+                        ptx::tmem_ld16(lane_addr + (uint32_t)(accbase * NT + cb), v);
+#pragma unroll
+                        for (int a = 1; a < NACC; ++a) {
+                            ptx::tmem_ld16(lane_addr + (uint32_t)((accbase + a) * NT + cb), w);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) v[i] += w[i];
+                        }
+                        if (row < L) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int o = o0 + cb + i;
+                                const long long idx = obase + (long long)o * Lout + t;
+                                float y = v[i] + __ldg(J.bias + o);
+                                if (MODE == MODE_AMP && J.res) y += J.res[idx];
+                                J.out[idx] = y;
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 0) ptx::tmem_dealloc(tmem, NCOLS);
+}
+
+// ----------------------------------------------------------------------------------------------
+// GEMM-only variant for the AMP convolutions: the activation has already been written to
+// memory as the A operand (rows of 8 bf16 channels, heads and tails in separate arrays, with
+// the conv's zero padding materialised), so both operands arrive by 1-D bulk copies and the
+// kernel needs only the MMA warp, the loader warp and 4 epilogue warps.
+// ----------------------------------------------------------------------------------------------
+
+constexpr int GEMM_THREADS = 192;   // warp 0 MMA, warp 1 loader, warps 2..5 epilogue
+
+struct GemmJob {
+    const uint8_t* a_hi;   // [B, Cin/8, Lpad] rows of 16 bytes
+    const uint8_t* a_lo;
+    const uint16_t* w;     // pre-split operand blocks
+    const float* bias;
+    const float* res;
+    float* out;
+    int K, dil, pad;
+};
+
+struct GemmParams {
+    GemmJob job[MH3A_MAX_RESBLOCKS];
+    int Cin, Cout, L, B, tiles_t;
+    int pad_l;            // zero rows before the sequence in the A arrays
+    long long Lpad;       // rows per (item, channel group) in the A arrays
+    int* err;
+};
+
+template <int MT, int NT, int NACC>
+__global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p, const TcPlan pl) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr int NHH = NACC - 1;
+    constexpr int USED = MT * NT * NACC;
+    static_assert(NACC >= 2 && USED <= 512, "tensor memory holds 512 columns");
+    constexpr int NCOLS = (USED <= 32) ? 32 : (USED <= 64) ? 64 : (USED <= 128) ? 128 : (USED <= 256) ? 256 : 512;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const GemmJob& J = p.job[blockIdx.z];
+    const int K = J.K, dil = J.dil, pad = J.pad;
+    const int Cin = p.Cin, Cout = p.Cout, L = p.L;
+    const int b = blockIdx.x / p.tiles_t;
+    const int t0 = (blockIdx.x % p.tiles_t) * (128 * MT);
+    const int o_tile = blockIdx.y;
+    const int o0 = o_tile * NT;
+    const int nchunks = Cin / KC;
+    const int ROWS = 128 * MT + (K - 1) * dil;
+    const int RS = pl.RS;
+
+    uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
+    uint8_t* Bs = smem + pl.offB;              // [NSB][2][KG][NT][16 B]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
+    uint64_t* a_full = bars;
+    uint64_t* a_empty = bars + NSA;
+    uint64_t* b_full = bars + 2 * NSA;
+    uint64_t* b_empty = bars + 2 * NSA + NSB;
+    uint64_t* acc_full = bars + 2 * NSA + 2 * NSB;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSA + 2 * NSB + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* epi_go = abort_flag + 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSA; ++s) {
+            ptx::mbar_init(&a_full[s], 1);
+            ptx::mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < NSB; ++s) {
+            ptx::mbar_init(&b_full[s], 1);
+            ptx::mbar_init(&b_empty[s], 1);
+        }
+        ptx::mbar_init(acc_full, 1);
+        *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+        *epi_go = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, NCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16(128, NT);
+            const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
+            const bool skip = *abort_flag != 0;
+            bool ok = !skip;
+            int u = 0;
+            for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
+                const int sa = chunk % NSA;
+                if (!ptx::mbar_wait(&a_full[sa], (chunk / NSA) & 1, kWaitLimit)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t a_hi = a_smem + sa * pl.SA;
+                const uint32_t a_lo = a_hi + KG * RS * 16;
+                for (int tap = 0; tap < K; ++tap, ++u) {
+                    const int sb = u % NSB;
+                    if (!ptx::mbar_wait(&b_full[sb], (u / NSB) & 1, kWaitLimit)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t b_hi = b_smem + sb * pl.SB;
+                    const uint32_t b_lo = b_hi + KG * NT * 16;
+#pragma unroll
+                    for (int kk = 0; kk < KG / 2; ++kk) {
+                        const uint32_t boff = (uint32_t)(2 * kk) * NT * 16;
+                        const uint64_t bh = ptx::smem_desc(b_hi + boff, NT * 16, 128);
+                        const uint64_t bl = ptx::smem_desc(b_lo + boff, NT * 16, 128);
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + tap * dil) * 16;
+                            const uint64_t ah = ptx::smem_desc(a_hi + aoff, RS * 16, 128);
+                            const uint64_t al = ptx::smem_desc(a_lo + aoff, RS * 16, 128);
+                            const int accbase = mt * NACC;
+                            const uint32_t dh = tmem + (uint32_t)((accbase + chunk % NHH) * NT);
+                            const uint32_t dx = tmem + (uint32_t)((accbase + NHH) * NT);
+                            const uint32_t acc_h = (chunk >= NHH || tap > 0 || kk > 0) ? 1u : 0u;
+                            const uint32_t acc_x = (chunk > 0 || tap > 0 || kk > 0) ? 1u : 0u;
+                            ptx::mma_bf16(dh, ah, bh, idesc, acc_h);
+                            ptx::mma_bf16(dx, ah, bl, idesc, acc_x);
+                            ptx::mma_bf16(dx, al, bh, idesc, 1u);
+                        }
+                    }
+                    ptx::mma_commit(&b_empty[sb]);
+                }
+                if (ok) ptx::mma_commit(&a_empty[sa]);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                if (!skip) atomicExch(p.err, 5);
+            }
+            ptx::mma_commit(acc_full);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- A and B loader
+        if (lane == 0) {
+            const size_t unit_elems = (size_t)2 * KG * NT * 8;
+            const uint16_t* wsrc = J.w + (size_t)o_tile * nchunks * K * unit_elems;
+            const uint32_t a_bytes = (uint32_t)(2 * KG * ROWS * 16);
+            const long long row0 = p.pad_l + t0 - pad;   // first window row in the A arrays
+            int a_issued = 0, b_issued = 0, u = 0;
+            bool ok = *abort_flag == 0;
+            for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
+                const int sa = chunk % NSA;
+                if (!ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                ptx::mbar_arrive_expect_tx(&a_full[sa], a_bytes);
+                for (int part = 0; part < 2; ++part) {
+                    const uint8_t* base = part == 0 ? J.a_hi : J.a_lo;
+                    for (int g = 0; g < KG; ++g) {
+                        const long long grp = (long long)b * (Cin / 8) + chunk * KG + g;
+                        ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KG + g) * RS) * 16,
+                                      base + (grp * p.Lpad + row0) * 16, (uint32_t)(ROWS * 16), &a_full[sa]);
+                    }
+                }
+                a_issued = chunk + 1;
+                for (int tap = 0; tap < K; ++tap, ++u) {
+                    const int sb = u % NSB;
+                    if (!ptx::mbar_wait(&b_empty[sb], ((u / NSB) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&b_full[sb], (uint32_t)pl.SB);
+                    ptx::bulk_g2s(Bs + (size_t)sb * pl.SB, wsrc + (size_t)u * unit_elems, (uint32_t)pl.SB, &b_full[sb]);
+                    b_issued = u + 1;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(p.err, 6);
+                // let the copies already in flight land before the CTA can exit
+                for (int c = (a_issued > NSA ? a_issued - NSA : 0); c < a_issued; ++c)
+                    ptx::mbar_wait(&a_full[c % NSA], (c / NSA) & 1, kWaitLimit);
+                for (int v = (b_issued > NSB ? b_issued - NSB : 0); v < b_issued; ++v)
+                    ptx::mbar_wait(&b_full[v % NSB], (v / NSB) & 1, kWaitLimit);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2..5)
+        if (threadIdx.x == 64) {
+            bool go = ptx::mbar_wait(acc_full, 0, kWaitLimit);
+            if (!go) atomicExch(p.err, 7);
+            go = go && *abort_flag == 0;
+            *epi_go = go ? 1 : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool go = *epi_go != 0;   // identical in all four epilogue warps
+        ptx::tc_fence_after();
+        const int q4 = warp & 3;        // TMEM lane quarter this warp may access
+        const long long obase = (long long)b * Cout * L;
+        if (go) {
+            const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int t = t0 + mt * 128 + q4 * 32 + lane;
-                for (int cb = part * CPP; cb < part * CPP + CPP && cb < NT; cb += 16) {
+                for (int cb = 0; cb < NT; cb += 16) {
                     float v[16], w[16];
-                    const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
                     ptx::tmem_ld16(lane_addr + (uint32_t)(mt * NACC * NT + cb), v);
 #pragma unroll
                     for (int a = 1; a < NACC; ++a) {
@@ -424,51 +726,158 @@ float bf16_value(uint16_t h) {
     return v;
 }
 
-int ntile_for(int C) { return C >= 256 ? 256 : C; }
+// Output-channel tile of each layer kind (the weight blocks are laid out for it).
+int ntile_amp(int C) { return C >= 64 ? 64 : C; }
+int ntile_pre(int) { return 64; }
+int ntile_convt(int Cout, int r) {
+    if (r > 2) return Cout >= 32 ? 32 : Cout;
+    return Cout >= 64 ? 64 : Cout;
+}
 
-template <int MT, int NT>
+template <int MODE, int MT, int NT, int NIN>
 TcPlan make_plan(const TcParams& p, int njobs) {
     int span = 0;
-    for (int j = 0; j < njobs; ++j) span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
+    if (MODE == MODE_CONVT) {
+        // tap shifts (phi + pad - j) / r + lo span [0, span]
+        const int K = p.job[0].K, pad = p.job[0].pad, r = p.r;
+        int smax = -1000000, smin = 1000000;
+        for (int j = 0; j < K; ++j) {
+            const int phase = ((j - pad) % r + r) % r;
+            const int a = phase + pad - j;
+            const int s = a >= 0 ? a / r : -((-a + r - 1) / r);
+            smax = std::max(smax, s);
+            smin = std::min(smin, s);
+        }
+        span = smax - smin;
+    } else {
+        for (int j = 0; j < njobs; ++j) span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
+    }
     TcPlan pl{};
     pl.RS = 128 * MT + span;
     pl.XWs = pl.RS + 12;
-    pl.SWs = 2 * pl.RS + 12;  // even (8-byte rows) with room for the last row pair's reads
+    pl.SWs = (MODE == MODE_AMP) ? 2 * pl.RS + 12 : 0;   // even (8-byte rows), room for the last pair
     pl.SA = 2 * KG * pl.RS * 16;
     pl.SB = 2 * KG * NT * 16;
     pl.offB = NSA * pl.SA;
     pl.offX = pl.offB + NSB * pl.SB;
-    const int stage_bytes = 8 * (2 * pl.XWs + pl.SWs) * 4;
+    const int stage_bytes = (2 * NIN * 8 * pl.XWs + 8 * pl.SWs) * 4;
     pl.offBar = (pl.offX + stage_bytes + 15) / 16 * 16;
     pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
     return pl;
 }
 
-template <int MT, int NT, int NACC>
+template <int MODE, int MT, int NT, int NACC, int R>
 int launch_tc(const TcParams& p0, int njobs, cudaStream_t s) {
     TcParams p = p0;
-    if (NACC - 1 > p.C / KC) return -1;  // every head accumulator must receive a chunk
+    if (NACC - 1 > p.Cin / KC) return -1;  // every head accumulator must receive a chunk
+    if (p.Cin % KC != 0 || p.Cout % NT != 0) return -1;
+    if (MODE == MODE_CONVT && p.r != R) return -1;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
-    const TcPlan pl = make_plan<MT, NT>(p, njobs);
+    constexpr int NIN = (MODE == MODE_CONVT) ? 3 : 1;
+    const TcPlan pl = make_plan<MODE, MT, NT, NIN>(p, njobs);
     if (pl.smem > 227 * 1024) return -1;
-    auto kern = k_amp_conv_tc<MT, NT, NACC>;
+    auto kern = k_conv_tc<MODE, MT, NT, NACC, R>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess) return -1;
-    dim3 grid(p.tiles_t * p.B, p.C / NT, njobs);
+    dim3 grid(p.tiles_t * p.B, p.Cout / NT, njobs);
     kern<<<grid, NTHREADS, pl.smem, s>>>(p, pl);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
 
-// Tile shape per width: MT x 128 time rows, NT output channels, NACC accumulators per M tile
-// (MT * NT * NACC <= 512 tensor-memory columns).
-int dispatch_tc(const TcParams& p, int njobs, cudaStream_t s) {
-    switch (p.C) {
-        case 512: return launch_tc<1, 256, 2>(p, njobs, s);
-        case 256: return launch_tc<1, 256, 2>(p, njobs, s);
-        case 128: return launch_tc<2, 128, 2>(p, njobs, s);
-        case 64: return launch_tc<2, 64, 3>(p, njobs, s);
-        case 32: return launch_tc<2, 32, 2>(p, njobs, s);
+// AMP tile shape per width: MT x 128 time rows, NT output channels, NACC accumulators per
+// M tile (MT * NT * NACC <= 512 tensor-memory columns).  The two widest stages use 128-column
+// tiles so that three head accumulators share their long K loops (accuracy: the accumulation
+// bias of these stages dominated the decode error with a single head accumulator).
+int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
+    switch (p.Cin) {
+        case 512: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
+        case 256: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
+        case 128: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
+        case 64: return launch_tc<MODE_AMP, 2, 64, 3, 1>(p, njobs, s);
+        case 32: return launch_tc<MODE_AMP, 2, 32, 2, 1>(p, njobs, s);
         default: return -1;
     }
+}
+
+template <int MT, int NT, int NACC>
+int launch_gemm(const GemmParams& p0, int njobs, cudaStream_t s) {
+    GemmParams p = p0;
+    if (NACC - 1 > p.Cin / KC || p.Cin % KC != 0 || p.Cout % NT != 0) return -1;
+    p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
+    int span = 0, padmax = 0;
+    for (int j = 0; j < njobs; ++j) {
+        span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
+        padmax = std::max(padmax, p.job[j].pad);
+    }
+    // every window row the tiles touch must exist in the A arrays
+    if (p.pad_l < padmax || p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax) return -1;
+    TcPlan pl{};
+    pl.RS = 128 * MT + span;
+    pl.SA = 2 * KG * pl.RS * 16;
+    pl.SB = 2 * KG * NT * 16;
+    pl.offB = NSA * pl.SA;
+    pl.offBar = (pl.offB + NSB * pl.SB + 15) / 16 * 16;
+    pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
+    if (pl.smem > 227 * 1024) return -1;
+    auto kern = k_gemm_tc<MT, NT, NACC>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess) return -1;
+    dim3 grid(p.tiles_t * p.B, p.Cout / NT, njobs);
+    kern<<<grid, GEMM_THREADS, pl.smem, s>>>(p, pl);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
+
+// GEMM tile shape per width (NT must match the weight packing of ntile_amp).
+int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
+    switch (p.Cin) {
+        case 512: return launch_gemm<1, 64, 4>(p, njobs, s);
+        case 256: return launch_gemm<1, 64, 4>(p, njobs, s);
+        case 128: return launch_gemm<1, 64, 4>(p, njobs, s);
+        case 64: return launch_gemm<1, 64, 3>(p, njobs, s);
+        case 32: return launch_gemm<2, 32, 2>(p, njobs, s);
+        default: return -1;
+    }
+}
+
+// Operand blocks: [o_tile][chunk][tap][part (head, tail)][group][row o][8 channels] as bf16,
+// from weights given as w(o, c, tap).
+template <class W>
+void pack_blocks(W w, int Cout, int Cin, int K, int NT, TcConv* out) {
+    const int ntiles = Cout / NT, nchunks = Cin / KC;
+    const size_t n = (size_t)Cout * Cin * K * 2;  // bf16 elements (head + tail)
+    std::vector<uint16_t> buf(n);
+    size_t pos = 0;
+    for (int ot = 0; ot < ntiles; ++ot)
+        for (int chk = 0; chk < nchunks; ++chk)
+            for (int tap = 0; tap < K; ++tap)
+                for (int part = 0; part < 2; ++part)
+                    for (int g = 0; g < KG; ++g)
+                        for (int o = 0; o < NT; ++o)
+                            for (int e = 0; e < 8; ++e) {
+                                const float v = w(ot * NT + o, chk * KC + g * 8 + e, tap);
+                                const uint16_t hb = bf16_bits_rn(v);
+                                buf[pos++] = part == 0 ? hb : bf16_bits_rn(v - bf16_value(hb));
+                            }
+    out->staging.assign(n / 2, 0.f);
+    std::memcpy(out->staging.data(), buf.data(), n * sizeof(uint16_t));
+    out->cout = Cout;
+    out->cin = Cin;
+    out->k = K;
+}
+
+TcJob make_job(const ConvJob& J, const TcConv& tw) {
+    TcJob T{};
+    T.x0 = J.x0;
+    T.x1 = J.x1;
+    T.x2 = J.x2;
+    T.w = reinterpret_cast<const uint16_t*>(tw.dev);
+    T.bias = J.bias;
+    T.alpha = J.alpha;
+    T.inv_beta = J.inv_beta;
+    T.res = J.res;
+    T.out = J.out;
+    T.K = J.K;
+    T.dil = J.dil;
+    T.pad = J.pad;
+    return T;
 }
 
 }  // namespace
@@ -484,47 +893,47 @@ bool tc_stage_supported(int C, const mh3a_config& c) {
     return true;
 }
 
-// Operand blocks: [o_tile][chunk][tap][part (head, tail)][group][row o][8 channels] as bf16.
-void prepare_tc_conv(const std::vector<float>& w, int C, int k, TcConv* out) {
-    const int NT = ntile_for(C);
-    const int ntiles = C / NT, nchunks = C / KC;
-    const size_t n = (size_t)C * C * k * 2;  // bf16 elements (head + tail)
-    std::vector<uint16_t> buf(n);
-    size_t pos = 0;
-    for (int ot = 0; ot < ntiles; ++ot)
-        for (int ch = 0; ch < nchunks; ++ch)
-            for (int tap = 0; tap < k; ++tap)
-                for (int part = 0; part < 2; ++part)
-                    for (int g = 0; g < KG; ++g)
-                        for (int o = 0; o < NT; ++o)
-                            for (int e = 0; e < 8; ++e) {
-                                const int oo = ot * NT + o, cc = ch * KC + g * 8 + e;
-                                const float v = w[((size_t)oo * C + cc) * k + tap];
-                                const uint16_t hb = bf16_bits_rn(v);
-                                buf[pos++] = part == 0 ? hb : bf16_bits_rn(v - bf16_value(hb));
-                            }
-    out->staging.assign(n / 2, 0.f);
-    std::memcpy(out->staging.data(), buf.data(), n * sizeof(uint16_t));
-    out->cout = C;
-    out->cin = C;
-    out->k = k;
+bool tc_pre_supported(int Cout, int Cin, int k) { return Cout % 64 == 0 && Cin % KC == 0 && Cin >= 7 * KC && k <= 15; }
+
+bool tc_convt_supported(int Cin, int Cout, int r, int K) {
+    if (Cin % KC != 0) return false;
+    if (r != 5 && r != 2) return false;
+    if (K > 16) return false;
+    const int NT = ntile_convt(Cout, r);
+    if (NT < 16 || NT % 16 != 0 || Cout % NT != 0) return false;
+    return true;
 }
 
-void prepare_tc_pre(const std::vector<float>&, int, int, int, TcStageWeights*) {}
+void prepare_tc_conv(const std::vector<float>& w, int C, int k, TcConv* out) {
+    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * C + c) * k + tap]; }, C, C, k, ntile_amp(C), out);
+}
+
+void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWeights* out) {
+    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + c) * k + tap]; }, O, I, k, ntile_pre(O),
+                &out->pre);
+}
+
+void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
+    pack_blocks([&](int o, int c, int tap) { return w_iok[((size_t)c * Cout + o) * K + tap]; }, Cout, Cin, K,
+                ntile_convt(Cout, r), out);
+}
 
 void tc_finalize(TcStageWeights* w) {
     for (auto& a : w->conv)
         for (auto& b : a)
             for (auto& c : b) std::vector<float>().swap(c.staging);
     std::vector<float>().swap(w->pre.staging);
+    std::vector<float>().swap(w->ups.staging);
 }
 
 int launch_conv_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int m, int half, cudaStream_t s,
                    int* err) {
     TcParams p{};
-    p.C = cp.Cin;
+    p.Cin = cp.Cin;
+    p.Cout = cp.Cout;
     p.L = cp.L;
     p.B = cp.B;
+    p.r = 1;
     p.filt = cp.filt;
     p.err = err;
     // heaviest kernel first (blockIdx.z = 0), so the longest blocks start earliest
@@ -532,25 +941,109 @@ int launch_conv_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int
     for (int j = 0; j < njobs; ++j) order[j] = j;
     std::sort(order, order + njobs, [&](int a, int b) { return cp.job[a].K > cp.job[b].K; });
     for (int z = 0; z < njobs; ++z) {
-        const int j = order[z];
-        const ConvJob& J = cp.job[j];
-        const TcConv& tw = w.conv[j][m][half];
+        const TcConv& tw = w.conv[order[z]][m][half];
         if (!tw.dev) return -1;
-        TcJob& T = p.job[z];
-        T.x = J.x0;
-        T.w = reinterpret_cast<const uint16_t*>(tw.dev);
-        T.bias = J.bias;
-        T.alpha = J.alpha;
-        T.inv_beta = J.inv_beta;
-        T.res = J.res;
-        T.out = J.out;
-        T.K = J.K;
-        T.dil = J.dil;
-        T.pad = J.pad;
+        p.job[z] = make_job(cp.job[order[z]], tw);
     }
-    return dispatch_tc(p, njobs, s);
+    return dispatch_amp(p, njobs, s);
 }
 
-int launch_conv_pre_tc(const ConvParams&, const TcStageWeights&, cudaStream_t) { return -1; }
+int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int m, int half,
+                       const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
+                       cudaStream_t s, int* err) {
+    GemmParams p{};
+    p.Cin = cp.Cin;
+    p.Cout = cp.Cout;
+    p.L = cp.L;
+    p.B = cp.B;
+    p.pad_l = pad_l;
+    p.Lpad = Lpad;
+    p.err = err;
+    // heaviest kernel first (blockIdx.z = 0), so the longest blocks start earliest
+    int order[MH3A_MAX_RESBLOCKS];
+    for (int j = 0; j < njobs; ++j) order[j] = j;
+    std::sort(order, order + njobs, [&](int a, int b) { return cp.job[a].K > cp.job[b].K; });
+    for (int z = 0; z < njobs; ++z) {
+        const int j = order[z];
+        const TcConv& tw = w.conv[j][m][half];
+        if (!tw.dev) return -1;
+        GemmJob& G = p.job[z];
+        G.a_hi = static_cast<const uint8_t*>(a_hi[j]);
+        G.a_lo = static_cast<const uint8_t*>(a_lo[j]);
+        G.w = reinterpret_cast<const uint16_t*>(tw.dev);
+        G.bias = cp.job[j].bias;
+        G.res = cp.job[j].res;
+        G.out = cp.job[j].out;
+        G.K = cp.job[j].K;
+        G.dil = cp.job[j].dil;
+        G.pad = cp.job[j].pad;
+    }
+    return dispatch_gemm(p, njobs, s);
+}
+
+int launch_conv_pre_tc(const ConvParams& cp, const TcStageWeights& w, cudaStream_t s, int* err) {
+    if (!w.pre.dev || cp.job[0].K > 15) return -1;
+    TcParams p{};
+    p.Cin = cp.Cin;
+    p.Cout = cp.Cout;
+    p.L = cp.L;
+    p.B = cp.B;
+    p.r = 1;
+    p.err = err;
+    p.job[0] = make_job(cp.job[0], w.pre);
+    // 7 head accumulators rotate over the 64 chunks of 2048 input channels
+    return launch_tc<MODE_PLAIN, 1, 64, 8, 1>(p, 1, s);
+}
+
+int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err) {
+    if (!w.ups.dev) return -1;
+    TcParams p{};
+    p.Cin = q.Cin;
+    p.Cout = q.Cout;
+    p.L = q.Lin;
+    p.B = q.B;
+    p.r = q.r;
+    p.err = err;
+    // window rows before the tile: minus the smallest tap shift floor((phi + pad - j) / r)
+    int smin = 1000000;
+    for (int j = 0; j < q.K; ++j) {
+        const int phase = ((j - q.pad) % q.r + q.r) % q.r;
+        const int a = phase + q.pad - j;
+        smin = std::min(smin, a >= 0 ? a / q.r : -((-a + q.r - 1) / q.r));
+    }
+    p.lo = -smin;
+    TcJob& T = p.job[0];
+    T.x0 = q.x0;
+    T.x1 = q.x1;
+    T.x2 = q.x2;
+    T.w = reinterpret_cast<const uint16_t*>(w.ups.dev);
+    T.bias = q.bias;
+    T.out = q.out;
+    T.K = q.K;
+    T.dil = 1;
+    T.pad = q.pad;
+    // as many head accumulators per phase as tensor memory (and the chunk count) allow
+    const int NT = ntile_convt(q.Cout, q.r);
+    const int nchunks = q.Cin / KC;
+    if (q.r == 5) {
+        switch (NT) {
+            case 32: return nchunks >= 2 ? launch_tc<MODE_CONVT, 1, 32, 3, 5>(p, 1, s)
+                                         : launch_tc<MODE_CONVT, 1, 32, 2, 5>(p, 1, s);
+            case 16: return launch_tc<MODE_CONVT, 1, 16, 2, 5>(p, 1, s);
+            default: return -1;
+        }
+    }
+    if (q.r == 2) {
+        switch (NT) {
+            case 128: return launch_tc<MODE_CONVT, 1, 128, 2, 2>(p, 1, s);
+            case 64: return nchunks >= 3 ? launch_tc<MODE_CONVT, 1, 64, 4, 2>(p, 1, s)
+                                         : launch_tc<MODE_CONVT, 1, 64, 2, 2>(p, 1, s);
+            case 32: return launch_tc<MODE_CONVT, 1, 32, 2, 2>(p, 1, s);
+            case 16: return launch_tc<MODE_CONVT, 1, 16, 2, 2>(p, 1, s);
+            default: return -1;
+        }
+    }
+    return -1;
+}
 
 }  // namespace mh3a

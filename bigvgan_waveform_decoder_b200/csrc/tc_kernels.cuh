@@ -16,15 +16,21 @@ struct TcConv {
 };
 
 struct TcStageWeights {
-    TcConv conv[MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS][2];
-    TcConv pre;
+    TcConv conv[MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS][2];  // AMP convs of the stage
+    TcConv ups;                                             // the stage's transposed conv
+    TcConv pre;                                             // conv_pre (stage 0 only)
 };
 
-// True when the AMP convolutions of a stage with C channels run on the tensor cores.
-bool tc_stage_supported(int C, const mh3a_config& c);
+// Which layers run on the tensor cores.
+bool tc_stage_supported(int C, const mh3a_config& c);           // AMP convs, C channels
+bool tc_pre_supported(int Cout, int Cin, int k);                 // conv_pre
+bool tc_convt_supported(int Cin, int Cout, int r, int K);        // transposed conv
 
+// Weight packing from folded fp32 weights: conv weights are [O, I, K], transposed-conv
+// weights [I, O, K].
 void prepare_tc_conv(const std::vector<float>& w_oik, int C, int k, TcConv* out);
 void prepare_tc_pre(const std::vector<float>& w_oik, int O, int I, int k, TcStageWeights* out);
+void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out);
 
 template <class AddFn>
 void tc_register(TcStageWeights* w, AddFn add) {
@@ -32,17 +38,26 @@ void tc_register(TcStageWeights* w, AddFn add) {
         for (auto& b : a)
             for (auto& c : b)
                 if (!c.staging.empty()) add(c.staging, &c.dev);
+    if (!w->ups.staging.empty()) add(w->ups.staging, &w->ups.dev);
     if (!w->pre.staging.empty()) add(w->pre.staging, &w->pre.dev);
 }
 
 // Drop host staging once the device copy exists.
 void tc_finalize(TcStageWeights* w);
 
-// Launch one AMP conv layer (dilation index m, half 0 = dilated conv, 1 = k x 1 conv) for all
-// residual blocks on the tensor cores.  Returns the number of kernels launched or -1.
-// `err` is a device int the kernel sets (non-zero) if one of its bounded waits times out.
+// Launchers; each returns the number of kernels launched or -1.  `err` is a device int the
+// kernels set (non-zero) if one of their bounded waits times out.
+// One AMP conv layer (dilation index m, half 0 = dilated conv, 1 = k x 1 conv) for all
+// residual blocks:
 int launch_conv_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int m, int half,
                    cudaStream_t s, int* err);
-int launch_conv_pre_tc(const ConvParams& p, const TcStageWeights& w, cudaStream_t s);
+// The same layer as a pure GEMM whose A operand (the activation, heads and tails) has been
+// written by launch_act_split into a_hi[j] / a_lo[j] with pad_l zero rows before the sequence
+// and Lpad rows per (item, channel group).
+int launch_amp_gemm_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int m, int half,
+                       const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
+                       cudaStream_t s, int* err);
+int launch_conv_pre_tc(const ConvParams& p, const TcStageWeights& w, cudaStream_t s, int* err);
+int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err);
 
 }  // namespace mh3a

@@ -177,6 +177,11 @@ MH3A_API mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int*
  * fp32 CUDA cores, -1 for a NULL handle or an out-of-range stage. */
 MH3A_API int mh3a_stage_uses_tensor_cores(const mh3a_handle* h, int stage);
 
+/* Same question per timing segment, numbered as in mh3a_segment_times: 0 input projection,
+ * 1 conv_pre, 2 + 2i upsampling stage i, 3 + 2i AMP stage i, 2 + 2 n_stages output conv.
+ * Returns 1, 0, or -1 for a NULL handle or an out-of-range segment. */
+MH3A_API int mh3a_segment_uses_tensor_cores(const mh3a_handle* h, int segment);
+
 /* Waits for the device, then reports whether any tensor-core kernel of this handle gave up
  * one of its bounded pipeline waits since the last check (MH3A_ERR_CUDA, with the reason in
  * mh3a_last_error(); the outputs of that call are invalid) and clears the flag.  Such a

@@ -59,7 +59,8 @@ def _decode_windows(dev, index, items):
             ref = oracle.decode(arch, w, z[b:b + 1, :, lo:hi], clamp=False)[0, 0]
             seg = ref[(klo - lo) * HOP:(khi - lo) * HOP]
             got = y[b, 0, klo * HOP:khi * HOP]
-            check(got, seg, Bd.MH3A_BF16X3, f"workload {index} item {b} frames {klo}-{khi}")
+            check(got, seg, Bd.MH3A_BF16X3, f"workload {index} item {b} frames {klo}-{khi}",
+                  waveform=True)
 
 
 def test_decode_10s_stereo_sampled(dev):
