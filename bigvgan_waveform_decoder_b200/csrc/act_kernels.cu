@@ -84,53 +84,91 @@ __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
         const int n_start = 2 * t0 - 5, SW = 2 * rows + 10;
         const float* xr0 = &xs[c][0] - xs_start;
         const int m_lo = n_start >> 1, m_hi = (n_start + SW - 1) >> 1;
-        for (int m = m_lo + lane; m <= m_hi; m += 32) {
-            const int mc = clampi(m, 0, L - 1);
-            float xv[7];
-#pragma unroll
-            for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
-            float ue = 0.f, uo = 0.f;
+        // u at both phases of position mc from x[mc-3 .. mc+3] (xv[k] = x[mc + k - 3 + off])
+        auto up2 = [&](const float* xv, int off, float& ue, float& uo) {
+            ue = 0.f;
+            uo = 0.f;
 #pragma unroll
             for (int k = 0; k < 6; ++k) {
-                ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
-                uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
+                ue = fmaf(p.filt.up[2 * k + 1], xv[off + 5 - k], ue);
+                uo = fmaf(p.filt.up[2 * k], xv[off + 6 - k], uo);
             }
-            const float se = fmaf(sin_sq_fast(al, ue), ib, ue);
-            const float so = fmaf(sin_sq_fast(al, uo), ib, uo);
-            const int ie = 2 * m - n_start;
-            if (ie >= 0 && ie < SW) sw[c][ie] = (m > L - 1) ? so : se;
-            if (ie + 1 >= 0 && ie + 1 < SW) sw[c][ie + 1] = (m < 0) ? se : so;
+        };
+        // A lane takes two consecutive input positions; inside the sequence they share eight
+        // inputs x[m0-3 .. m0+4].  At the ends each position is clamped on its own.
+        for (int m0 = m_lo + 2 * lane; m0 <= m_hi; m0 += 64) {
+            float ue[2], uo[2];
+            if (m0 >= 0 && m0 + 1 <= L - 1) {
+                float xv[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) xv[k] = xr0[m0 + k - 3];
+                up2(xv, 0, ue[0], uo[0]);
+                up2(xv, 1, ue[1], uo[1]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int mc = clampi(m0 + i, 0, L - 1);
+                    float xv[7];
+#pragma unroll
+                    for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
+                    up2(xv, 0, ue[i], uo[i]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int m = m0 + i;
+                if (m > m_hi) break;
+                const float se = fmaf(sin_sq_fast(al, ue[i]), ib, ue[i]);
+                const float so = fmaf(sin_sq_fast(al, uo[i]), ib, uo[i]);
+                const int ie = 2 * m - n_start;
+                if (ie >= 0 && ie < SW) sw[c][ie] = (m > L - 1) ? so : se;
+                if (ie + 1 >= 0 && ie + 1 < SW) sw[c][ie + 1] = (m < 0) ? se : so;
+            }
         }
     }
     __syncthreads();
-    // decimate, zero outside [0, L), split into head and tail, one 16-byte row per thread
-    for (int q = tid; q < rows; q += NT_ACT) {
-        const int t = t0 + q;
-        float a[8];
-        if (t >= 0 && t < L) {
+    // decimate, zero outside [0, L), split into head and tail: 2 rows x 4 channels per item
+    const int npairs = (rows + 1) >> 1;
+    for (int it = tid; it < 2 * npairs; it += NT_ACT) {
+        const int rp = it >> 1, hf = it & 1;
+        const int q0 = 2 * rp;
+        float a0[4], a1[4];
+        if (any_inside) {
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const float2* sr = reinterpret_cast<const float2*>(&sw[cc][2 * q]);
-                float v = 0.f;
+            for (int cc = 0; cc < 4; ++cc) {
+                const float2* sr = reinterpret_cast<const float2*>(&sw[4 * hf + cc][2 * q0]);
+                float s[14];
 #pragma unroll
-                for (int j = 0; j < kFilterTaps / 2; ++j) {
+                for (int j = 0; j < 7; ++j) {
                     const float2 s2 = sr[j];
-                    v = fmaf(p.filt.down[2 * j], s2.x, v);
-                    v = fmaf(p.filt.down[2 * j + 1], s2.y, v);
+                    s[2 * j] = s2.x;
+                    s[2 * j + 1] = s2.y;
                 }
-                a[cc] = v;
-            }
-        } else {
+                float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) a[cc] = 0.f;
+                for (int j = 0; j < kFilterTaps; ++j) {
+                    v0 = fmaf(p.filt.down[j], s[j], v0);
+                    v1 = fmaf(p.filt.down[j], s[j + 2], v1);
+                }
+                a0[cc] = v0;
+                a1[cc] = v1;
+            }
         }
-        uint4 hv, lv;
-        split2(a[0], a[1], &hv.x, &lv.x);
-        split2(a[2], a[3], &hv.y, &lv.y);
-        split2(a[4], a[5], &hv.z, &lv.z);
-        split2(a[6], a[7], &hv.w, &lv.w);
-        ohi[t] = hv;
-        olo[t] = lv;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int q = q0 + r;
+            if (q >= rows) break;
+            const int t = t0 + q;
+            const bool in = t >= 0 && t < L;
+            float v[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) v[cc] = in ? (r == 0 ? a0[cc] : a1[cc]) : 0.f;
+            uint2 hv, lv;
+            split2(v[0], v[1], &hv.x, &lv.x);
+            split2(v[2], v[3], &hv.y, &lv.y);
+            reinterpret_cast<uint2*>(ohi + t)[hf] = hv;
+            reinterpret_cast<uint2*>(olo + t)[hf] = lv;
+        }
     }
 }
 

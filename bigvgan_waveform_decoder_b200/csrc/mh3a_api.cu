@@ -491,8 +491,11 @@ mh3a_status amp_stage_into(mh3a_handle* h, const float* x, int B, int L, int sta
                 J.dil = d;
                 J.pad = d * (k - 1) / 2;
             }
-            const int n = h->stage_tc[stage] ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err)
-                                             : launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
+            // the fused tensor-core kernel (activation computed in its own producer warps) needs
+            // no operand buffers beyond X and T; it serves widths of 32 channels and more
+            const int n = (h->stage_tc[stage] && C >= 32)
+                              ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err)
+                              : launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             mh3a_status st = counted(h, n);
             if (st) return st;
         }

@@ -512,16 +512,24 @@ struct GemmParams {
     int Cin, Cout, L, B, tiles_t;
     int pad_l;            // zero rows before the sequence in the A arrays
     long long Lpad;       // rows per (item, channel group) in the A arrays
+    int tpu;              // tap units per weight bulk copy (set by the launcher)
     int* err;
 };
 
-template <int MT, int NT, int NACC>
+// KGT = 8-channel groups per K chunk (4: 32 input channels; 2: 16).  KGT = 1 serves 8-channel
+// layers: one MMA K-step of 16 then covers the same 8 channels at two consecutive taps -- the
+// second core matrix along K is the window shifted by `dil` rows, i.e. the A descriptor's
+// leading-byte offset is dil * 16 -- and the weight block of a unit holds that tap pair (a
+// zero block stands in for the tap past the last one).
+template <int MT, int NT, int NACC, int KGT>
 __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p, const TcPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int NHH = NACC - 1;
     constexpr int USED = MT * NT * NACC;
     static_assert(NACC >= 2 && USED <= 512, "tensor memory holds 512 columns");
+    static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
     constexpr int NCOLS = (USED <= 32) ? 32 : (USED <= 64) ? 64 : (USED <= 128) ? 128 : (USED <= 256) ? 256 : 512;
+    constexpr int BG = (KGT == 1) ? 2 : KGT;   // core-matrix columns (K) per weight block part
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const GemmJob& J = p.job[blockIdx.z];
     const int K = J.K, dil = J.dil, pad = J.pad;
@@ -530,8 +538,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
     const int t0 = (blockIdx.x % p.tiles_t) * (128 * MT);
     const int o_tile = blockIdx.y;
     const int o0 = o_tile * NT;
-    const int nchunks = Cin / KC;
-    const int ROWS = 128 * MT + (K - 1) * dil;
+    const int nchunks = Cin / (8 * KGT);
+    const int KU = (KGT == 1) ? (K + 1) / 2 : K;            // tap units (taps or tap pairs) per chunk
+    const int TPU = p.tpu;                                   // tap units per weight copy
+    const int NUC = (KU + TPU - 1) / TPU;                    // weight copies per chunk
+    constexpr int TAPB = 2 * BG * NT * 16;                   // bytes of one tap unit (head + tail)
+    const int ROWS = 128 * MT + (K - 1) * dil + (KGT == 1 ? dil : 0);
     const int RS = pl.RS;
 
     uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
@@ -582,32 +594,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
                 if (!ptx::mbar_wait(&a_full[sa], (chunk / NSA) & 1, kWaitLimit)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t a_hi = a_smem + sa * pl.SA;
-                const uint32_t a_lo = a_hi + KG * RS * 16;
-                for (int tap = 0; tap < K; ++tap, ++u) {
+                const uint32_t a_lo = a_hi + KGT * RS * 16;
+                for (int uc = 0; uc < NUC; ++uc, ++u) {
                     const int sb = u % NSB;
                     if (!ptx::mbar_wait(&b_full[sb], (u / NSB) & 1, kWaitLimit)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t b_hi = b_smem + sb * pl.SB;
-                    const uint32_t b_lo = b_hi + KG * NT * 16;
+                    const int ut_end = min(KU, (uc + 1) * TPU);
+                    for (int unit = uc * TPU; unit < ut_end; ++unit) {
+                    const uint32_t b_hi = b_smem + sb * pl.SB + (unit - uc * TPU) * TAPB;
+                    const uint32_t b_lo = b_hi + BG * NT * 16;
+                    // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
+                    // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
+                    const int row_shift = (KGT == 1 ? 2 * unit : unit) * dil;
+                    const uint32_t a_lbo = (KGT == 1) ? (uint32_t)dil * 16 : (uint32_t)RS * 16;
 #pragma unroll
-                    for (int kk = 0; kk < KG / 2; ++kk) {
+                    for (int kk = 0; kk < (KGT == 1 ? 1 : KGT / 2); ++kk) {
                         const uint32_t boff = (uint32_t)(2 * kk) * NT * 16;
                         const uint64_t bh = ptx::smem_desc(b_hi + boff, NT * 16, 128);
                         const uint64_t bl = ptx::smem_desc(b_lo + boff, NT * 16, 128);
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
-                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + tap * dil) * 16;
-                            const uint64_t ah = ptx::smem_desc(a_hi + aoff, RS * 16, 128);
-                            const uint64_t al = ptx::smem_desc(a_lo + aoff, RS * 16, 128);
+                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + row_shift) * 16;
+                            const uint64_t ah = ptx::smem_desc(a_hi + aoff, a_lbo, 128);
+                            const uint64_t al = ptx::smem_desc(a_lo + aoff, a_lbo, 128);
                             const int accbase = mt * NACC;
                             const uint32_t dh = tmem + (uint32_t)((accbase + chunk % NHH) * NT);
                             const uint32_t dx = tmem + (uint32_t)((accbase + NHH) * NT);
-                            const uint32_t acc_h = (chunk >= NHH || tap > 0 || kk > 0) ? 1u : 0u;
-                            const uint32_t acc_x = (chunk > 0 || tap > 0 || kk > 0) ? 1u : 0u;
+                            const uint32_t acc_h = (chunk >= NHH || unit > 0 || kk > 0) ? 1u : 0u;
+                            const uint32_t acc_x = (chunk > 0 || unit > 0 || kk > 0) ? 1u : 0u;
                             ptx::mma_bf16(dh, ah, bh, idesc, acc_h);
                             ptx::mma_bf16(dx, ah, bl, idesc, acc_x);
                             ptx::mma_bf16(dx, al, bh, idesc, 1u);
                         }
+                    }
                     }
                     ptx::mma_commit(&b_empty[sb]);
                 }
@@ -623,9 +642,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
     } else if (warp == 1) {
         // ---------------------------------------------------------------- A and B loader
         if (lane == 0) {
-            const size_t unit_elems = (size_t)2 * KG * NT * 8;
-            const uint16_t* wsrc = J.w + (size_t)o_tile * nchunks * K * unit_elems;
-            const uint32_t a_bytes = (uint32_t)(2 * KG * ROWS * 16);
+            const size_t unit_elems = (size_t)2 * BG * NT * 8;
+            const uint16_t* wsrc = J.w + (size_t)o_tile * nchunks * KU * unit_elems;
+            const uint32_t a_bytes = (uint32_t)(2 * KGT * ROWS * 16);
             const long long row0 = p.pad_l + t0 - pad;   // first window row in the A arrays
             int a_issued = 0, b_issued = 0, u = 0;
             bool ok = *abort_flag == 0;
@@ -635,18 +654,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
                 ptx::mbar_arrive_expect_tx(&a_full[sa], a_bytes);
                 for (int part = 0; part < 2; ++part) {
                     const uint8_t* base = part == 0 ? J.a_hi : J.a_lo;
-                    for (int g = 0; g < KG; ++g) {
-                        const long long grp = (long long)b * (Cin / 8) + chunk * KG + g;
-                        ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KG + g) * RS) * 16,
+                    for (int g = 0; g < KGT; ++g) {
+                        const long long grp = (long long)b * (Cin / 8) + chunk * KGT + g;
+                        ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KGT + g) * RS) * 16,
                                       base + (grp * p.Lpad + row0) * 16, (uint32_t)(ROWS * 16), &a_full[sa]);
                     }
                 }
                 a_issued = chunk + 1;
-                for (int tap = 0; tap < K; ++tap, ++u) {
+                for (int uc = 0; uc < NUC; ++uc, ++u) {
                     const int sb = u % NSB;
                     if (!ptx::mbar_wait(&b_empty[sb], ((u / NSB) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&b_full[sb], (uint32_t)pl.SB);
-                    ptx::bulk_g2s(Bs + (size_t)sb * pl.SB, wsrc + (size_t)u * unit_elems, (uint32_t)pl.SB, &b_full[sb]);
+                    // tap units [uc * TPU, min(KU, (uc + 1) * TPU)) are contiguous in the packing
+                    const int nunits = min(KU, (uc + 1) * TPU) - uc * TPU;
+                    const uint32_t bytes = (uint32_t)(nunits * TAPB);
+                    ptx::mbar_arrive_expect_tx(&b_full[sb], bytes);
+                    ptx::bulk_g2s(Bs + (size_t)sb * pl.SB, wsrc + ((size_t)chunk * KU + (size_t)uc * TPU) * unit_elems,
+                                  bytes, &b_full[sb]);
                     b_issued = u + 1;
                 }
             }
@@ -692,6 +715,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int o = o0 + cb + i;
+                            if (o >= Cout) break;   // output channels padded up to the tile width
                             const long long idx = obase + (long long)o * L + t;
                             float y = v[i] + __ldg(J.bias + o);
                             if (J.res) y += J.res[idx];
@@ -798,65 +822,102 @@ int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
     }
 }
 
-template <int MT, int NT, int NACC>
+template <int MT, int NT, int NACC, int KGT>
 int launch_gemm(const GemmParams& p0, int njobs, cudaStream_t s) {
     GemmParams p = p0;
-    if (NACC - 1 > p.Cin / KC || p.Cin % KC != 0 || p.Cout % NT != 0) return -1;
+    const int kc = 8 * KGT;
+    if (NACC - 1 > p.Cin / kc || p.Cin % kc != 0) return -1;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
-    int span = 0, padmax = 0;
+    int span = 0, padmax = 0, dilmax = 0;
     for (int j = 0; j < njobs; ++j) {
         span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
         padmax = std::max(padmax, p.job[j].pad);
+        dilmax = std::max(dilmax, p.job[j].dil);
     }
+    const int extra = (KGT == 1) ? dilmax : 0;   // the phantom tap of the last tap pair
     // every window row the tiles touch must exist in the A arrays
-    if (p.pad_l < padmax || p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax) return -1;
+    if (p.pad_l < padmax ||
+        p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax + extra)
+        return -1;
+    // weight copies of about 16 KB: one L2 round trip then feeds several taps' MMAs
+    constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * NT * 16;
+    int kumax = 1;
+    for (int j = 0; j < njobs; ++j) kumax = std::max(kumax, KGT == 1 ? (p.job[j].K + 1) / 2 : p.job[j].K);
+    p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));
     TcPlan pl{};
-    pl.RS = 128 * MT + span;
-    pl.SA = 2 * KG * pl.RS * 16;
-    pl.SB = 2 * KG * NT * 16;
+    pl.RS = 128 * MT + span + extra;
+    pl.SA = 2 * KGT * pl.RS * 16;
+    // ... but not at the cost of the second CTA per SM (2 x 113 KB of shared memory)
+    while (p.tpu > 1 && NSA * pl.SA + NSB * p.tpu * TAPB + 1024 > 113 * 1024) --p.tpu;
+    pl.SB = p.tpu * TAPB;
     pl.offB = NSA * pl.SA;
     pl.offBar = (pl.offB + NSB * pl.SB + 15) / 16 * 16;
     pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
     if (pl.smem > 227 * 1024) return -1;
-    auto kern = k_gemm_tc<MT, NT, NACC>;
+    auto kern = k_gemm_tc<MT, NT, NACC, KGT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess) return -1;
-    dim3 grid(p.tiles_t * p.B, p.Cout / NT, njobs);
+    dim3 grid(p.tiles_t * p.B, (p.Cout + NT - 1) / NT, njobs);
     kern<<<grid, GEMM_THREADS, pl.smem, s>>>(p, pl);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
 
-// GEMM tile shape per width (NT must match the weight packing of ntile_amp).
+// GEMM tile shape per width; NT and the channels per chunk must match amp_layout().
 int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_gemm<1, 64, 4>(p, njobs, s);
-        case 256: return launch_gemm<1, 64, 4>(p, njobs, s);
-        case 128: return launch_gemm<1, 64, 4>(p, njobs, s);
-        case 64: return launch_gemm<1, 64, 3>(p, njobs, s);
-        case 32: return launch_gemm<2, 32, 2>(p, njobs, s);
+        case 512: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
+        case 256: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
+        case 128: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
+        case 64: return launch_gemm<1, 64, 3, 4>(p, njobs, s);
+        case 32: return launch_gemm<2, 32, 2, 4>(p, njobs, s);
+        case 16: return launch_gemm<2, 16, 2, 2>(p, njobs, s);
+        case 8: return launch_gemm<2, 16, 2, 1>(p, njobs, s);
         default: return -1;
     }
 }
 
-// Operand blocks: [o_tile][chunk][tap][part (head, tail)][group][row o][8 channels] as bf16,
-// from weights given as w(o, c, tap).
+// Weight-block layout of the AMP convolutions by width: output tile NT and 8-channel groups
+// per K chunk (1 = tap-pair units for 8-channel layers).
+void amp_layout(int C, int* NT, int* KGT) {
+    if (C >= 32) {
+        *NT = ntile_amp(C);
+        *KGT = 4;
+    } else if (C == 16) {
+        *NT = 16;
+        *KGT = 2;
+    } else {
+        *NT = 16;
+        *KGT = 1;
+    }
+}
+
+// Operand blocks: [o_tile][chunk][unit][part (head, tail)][core column][row o][8 channels] as
+// bf16, from weights given as w(o, c, tap).  For KGT >= 2 a unit is one tap and the core
+// columns are the chunk's channel groups; for KGT == 1 a unit is a tap pair and the two core
+// columns are its taps (zero past the last tap).  Rows o >= Cout are zero.
 template <class W>
-void pack_blocks(W w, int Cout, int Cin, int K, int NT, TcConv* out) {
-    const int ntiles = Cout / NT, nchunks = Cin / KC;
-    const size_t n = (size_t)Cout * Cin * K * 2;  // bf16 elements (head + tail)
+void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, TcConv* out) {
+    const int kc = 8 * KGT;
+    const int ntiles = (Cout + NT - 1) / NT, nchunks = Cin / kc;
+    const int KU = (KGT == 1) ? (K + 1) / 2 : K;
+    const int BG = (KGT == 1) ? 2 : KGT;
+    const size_t n = (size_t)ntiles * nchunks * KU * 2 * BG * NT * 8;  // bf16 elements
     std::vector<uint16_t> buf(n);
     size_t pos = 0;
     for (int ot = 0; ot < ntiles; ++ot)
         for (int chk = 0; chk < nchunks; ++chk)
-            for (int tap = 0; tap < K; ++tap)
+            for (int unit = 0; unit < KU; ++unit)
                 for (int part = 0; part < 2; ++part)
-                    for (int g = 0; g < KG; ++g)
+                    for (int col = 0; col < BG; ++col)
                         for (int o = 0; o < NT; ++o)
                             for (int e = 0; e < 8; ++e) {
-                                const float v = w(ot * NT + o, chk * KC + g * 8 + e, tap);
+                                const int oo = ot * NT + o;
+                                const int tap = (KGT == 1) ? 2 * unit + col : unit;
+                                const int cc = chk * kc + ((KGT == 1) ? 0 : col * 8) + e;
+                                const float v = (oo < Cout && tap < K) ? w(oo, cc, tap) : 0.f;
                                 const uint16_t hb = bf16_bits_rn(v);
                                 buf[pos++] = part == 0 ? hb : bf16_bits_rn(v - bf16_value(hb));
                             }
-    out->staging.assign(n / 2, 0.f);
+    out->staging.assign((n + 1) / 2, 0.f);
     std::memcpy(out->staging.data(), buf.data(), n * sizeof(uint16_t));
     out->cout = Cout;
     out->cin = Cin;
@@ -883,7 +944,7 @@ TcJob make_job(const ConvJob& J, const TcConv& tw) {
 }  // namespace
 
 bool tc_stage_supported(int C, const mh3a_config& c) {
-    if (C != 512 && C != 256 && C != 128 && C != 64 && C != 32) return false;
+    if (C != 512 && C != 256 && C != 128 && C != 64 && C != 32 && C != 16 && C != 8) return false;
     if (c.n_resblocks != 3) return false;
     for (int j = 0; j < c.n_resblocks; ++j)
         for (int m = 0; m < c.n_dilations; ++m) {
@@ -905,17 +966,19 @@ bool tc_convt_supported(int Cin, int Cout, int r, int K) {
 }
 
 void prepare_tc_conv(const std::vector<float>& w, int C, int k, TcConv* out) {
-    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * C + c) * k + tap]; }, C, C, k, ntile_amp(C), out);
+    int NT, KGT;
+    amp_layout(C, &NT, &KGT);
+    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * C + c) * k + tap]; }, C, C, k, NT, KGT, out);
 }
 
 void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWeights* out) {
-    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + c) * k + tap]; }, O, I, k, ntile_pre(O),
+    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + c) * k + tap]; }, O, I, k, ntile_pre(O), KG,
                 &out->pre);
 }
 
 void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
     pack_blocks([&](int o, int c, int tap) { return w_iok[((size_t)c * Cout + o) * K + tap]; }, Cout, Cin, K,
-                ntile_convt(Cout, r), out);
+                ntile_convt(Cout, r), KG, out);
 }
 
 void tc_finalize(TcStageWeights* w) {
