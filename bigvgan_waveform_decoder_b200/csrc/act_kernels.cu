@@ -13,6 +13,12 @@
 // tensor-core kernel copies straight into shared memory.  Rows [-pad_l, 0) and [L, L + pad_r)
 // are written as zeros: they are the conv's zero padding, so the GEMM never special-cases the
 // sequence ends.  Heads and tails go to separate arrays.
+//
+// A block covers TT = 512 output rows of one channel group.  Tiles away from the sequence ends
+// take the fast path: every lane owns 16 consecutive outputs of one channel, forms the 32
+// SnakeBeta values at the 2x rate that belong to them in registers, receives the 5 + 5 halo
+// values from its neighbour lanes by warp shuffles, and decimates in registers.  The tiles at
+// the ends take the general path, which clamps every index.
 #include <cuda_bf16.h>
 
 #include "act_kernels.cuh"
@@ -20,10 +26,23 @@
 namespace mh3a {
 namespace {
 
-constexpr int TT = 384;       // output rows per block (static shared memory stays under 48 KB)
-constexpr int NT_ACT = 256;   // threads per block (8 warps: one per channel of the group)
+constexpr int TT = 512;                   // output rows per block
+constexpr int RUN = 16;                   // outputs per lane on the fast path (TT = 32 RUN)
+constexpr int TG = 256;                   // rows per sub-tile of the general path
+constexpr int NT_ACT = 256;               // threads per block (8 warps: one per channel)
+constexpr int NS = 2 * RUN + 10;          // SnakeBeta values one lane's decimation reads
+// Fast-path shared layout: per channel a window of x and a row of outputs, each with 4 floats
+// of padding after every 16 so that lanes reading 16-float runs hit distinct banks.
+constexpr int XF = TT + 16;               // x[t0 - 8, t0 + TT + 8)
+constexpr int XF_P = XF + XF / 16 * 4;
+constexpr int TF_P = TT + TT / 16 * 4;
+// General-path shared layout.
+constexpr int XG = TG + 16;
+constexpr int SG = 2 * TG + 12;
+constexpr int SMEM_FLOATS = (8 * (XF_P + TF_P) > 8 * (XG + SG)) ? 8 * (XF_P + TF_P) : 8 * (XG + SG);
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+__device__ __forceinline__ int skew(int i) { return i + ((i >> 4) << 2); }
 
 // sin^2(alpha u): Cody-Waite reduction modulo pi, then the hardware sine on [-pi/2, pi/2]
 // (absolute error near 2^-21, far below the 3xBF16 operand error).
@@ -56,118 +75,182 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t* h, uint32_t* 
     *l = pack2(a - ha, b - hb);
 }
 
-// grid: x = row tiles over [-pad_l, L + pad_r), y = B * C / 8 (item, group), z = job
-__global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
-    __shared__ float xs[8][TT + 16];
-    __shared__ __align__(16) float sw[8][2 * TT + 12];
-    const ActJob& J = p.job[blockIdx.z];
-    const int C = p.C, L = p.L;
-    const int ngroups = C / 8;
-    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
-    const int t0 = -p.pad_l + blockIdx.x * TT;           // first output row of the tile
-    const int rows = min(TT, L + p.pad_r - t0);
-    const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
-    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
-    uint4* ohi = reinterpret_cast<uint4*>(J.a_hi) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
-    uint4* olo = reinterpret_cast<uint4*>(J.a_lo) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
+// ---------------------------------------------------------------------------------------------
+// fast path: rows [t0, t0 + TT) with 8 <= t0 and t0 + TT + 8 <= L, so that neither the input
+// window nor the 2x-rate SnakeBeta window reaches past a sequence end
+// ---------------------------------------------------------------------------------------------
 
+// SnakeBeta value j of a lane's window, n = 2 (t0 + q0) - 5 + j, from xv[k] = x[t0 + q0 - 8 + k]
+// (j even: odd phase n = 2m + 1; j odd: even phase n = 2m).
+template <int J>
+__device__ __forceinline__ float snake_at(const ActFilter& f, const float* xv, float al, float ib) {
+    float u = 0.f;
+    if (J % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k], xv[8 + J / 2 - k], u);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k + 1], xv[8 + (J - 1) / 2 - k], u);
+    }
+    return fmaf(sin_sq_fast(al, u), ib, u);
+}
+
+template <int J0, int J1>
+__device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv, float al, float ib, float* s) {
+    if constexpr (J0 < J1) {
+        s[J0] = snake_at<J0>(f, xv, al, ib);
+        snake_range<J0 + 1, J1>(f, xv, al, ib, s);
+    }
+}
+
+__device__ __forceinline__ void act_tile_fast(const ActParams& p, const ActJob& J, float* buf, int b,
+                                              int g, int t0, uint4* ohi, uint4* olo) {
+    const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
+    float* xs = buf + c * XF_P;
+    float* T = buf + 8 * XF_P;   // [8][TF_P] outputs, skewed
+    const float* xrow = J.x + ((long long)b * p.C + g * 8 + c) * p.L + (t0 - 8);
+    for (int i = lane; i < XF; i += 32) xs[skew(i)] = __ldg(xrow + i);
+    __syncwarp();
+    const float al = __ldg(J.alpha + g * 8 + c), ib = __ldg(J.inv_beta + g * 8 + c);
+    const int q0 = RUN * lane;
+    float xv[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(xs + skew(q0 + 4 * k));
+        xv[4 * k] = v.x;
+        xv[4 * k + 1] = v.y;
+        xv[4 * k + 2] = v.z;
+        xv[4 * k + 3] = v.w;
+    }
+    float s[NS];
+    snake_range<5, 5 + 2 * RUN>(p.filt, xv, al, ib, s);     // the lane's own 2 RUN values
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+        s[j] = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
+        s[j + 5 + 2 * RUN] = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
+    }
+    if (lane == 0) snake_range<0, 5>(p.filt, xv, al, ib, s);
+    if (lane == 31) snake_range<5 + 2 * RUN, NS>(p.filt, xv, al, ib, s);
+    float a[RUN];
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(p.filt.down[j], s[2 * i + j], v);
+        a[i] = v;
+    }
+    float* trow = T + c * TF_P;
+#pragma unroll
+    for (int k = 0; k < RUN / 4; ++k)
+        *reinterpret_cast<float4*>(trow + skew(q0 + 4 * k)) = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
+    __syncthreads();
+    for (int q = tid; q < TT; q += NT_ACT) {
+        const int qs = skew(q);
+        float v[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) v[cc] = T[cc * TF_P + qs];
+        uint4 hv, lv;
+        split2(v[0], v[1], &hv.x, &lv.x);
+        split2(v[2], v[3], &hv.y, &lv.y);
+        split2(v[4], v[5], &hv.z, &lv.z);
+        split2(v[6], v[7], &hv.w, &lv.w);
+        ohi[t0 + q] = hv;
+        olo[t0 + q] = lv;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// general path: rows [t0, t0 + rows), rows <= TG, anywhere in [-pad_l, L + pad_r)
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void act_tile_general(const ActParams& p, const ActJob& J, float* buf, int b,
+                                                 int g, int t0, int rows, uint4* ohi, uint4* olo) {
+    const int C = p.C, L = p.L;
+    const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
+    float* xs = buf;              // [8][XG]
+    float* sw = buf + 8 * XG;     // [8][SG]
     const bool any_inside = t0 < L && t0 + rows > 0;
     if (any_inside) {
         const int xs_start = t0 - 6;
         const int XW = rows + 12;
         const float* xrow = J.x + ((long long)b * C + g * 8 + c) * L;
-        for (int q = lane; q < XW; q += 32) xs[c][q] = __ldg(xrow + clampi(xs_start + q, 0, L - 1));
+        float* xc = xs + c * XG;
+        for (int q = lane; q < XW; q += 32) xc[q] = __ldg(xrow + clampi(xs_start + q, 0, L - 1));
         __syncwarp();
         // SnakeBeta at the 2x rate over n in [2 t0 - 5, 2 (t0 + rows) + 5): a lane takes one
         // input position m and forms both phases; positions past either end repeat the end.
         const float al = __ldg(J.alpha + g * 8 + c), ib = __ldg(J.inv_beta + g * 8 + c);
         const int n_start = 2 * t0 - 5, SW = 2 * rows + 10;
-        const float* xr0 = &xs[c][0] - xs_start;
+        const float* xr0 = xc - xs_start;
+        float* sc = sw + c * SG;
         const int m_lo = n_start >> 1, m_hi = (n_start + SW - 1) >> 1;
-        // u at both phases of position mc from x[mc-3 .. mc+3] (xv[k] = x[mc + k - 3 + off])
-        auto up2 = [&](const float* xv, int off, float& ue, float& uo) {
-            ue = 0.f;
-            uo = 0.f;
+        for (int m = m_lo + lane; m <= m_hi; m += 32) {
+            const int mc = clampi(m, 0, L - 1);
+            float xv[7];
+#pragma unroll
+            for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
+            float ue = 0.f, uo = 0.f;
 #pragma unroll
             for (int k = 0; k < 6; ++k) {
-                ue = fmaf(p.filt.up[2 * k + 1], xv[off + 5 - k], ue);
-                uo = fmaf(p.filt.up[2 * k], xv[off + 6 - k], uo);
+                ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
+                uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
             }
-        };
-        // A lane takes two consecutive input positions; inside the sequence they share eight
-        // inputs x[m0-3 .. m0+4].  At the ends each position is clamped on its own.
-        for (int m0 = m_lo + 2 * lane; m0 <= m_hi; m0 += 64) {
-            float ue[2], uo[2];
-            if (m0 >= 0 && m0 + 1 <= L - 1) {
-                float xv[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) xv[k] = xr0[m0 + k - 3];
-                up2(xv, 0, ue[0], uo[0]);
-                up2(xv, 1, ue[1], uo[1]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int mc = clampi(m0 + i, 0, L - 1);
-                    float xv[7];
-#pragma unroll
-                    for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
-                    up2(xv, 0, ue[i], uo[i]);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int m = m0 + i;
-                if (m > m_hi) break;
-                const float se = fmaf(sin_sq_fast(al, ue[i]), ib, ue[i]);
-                const float so = fmaf(sin_sq_fast(al, uo[i]), ib, uo[i]);
-                const int ie = 2 * m - n_start;
-                if (ie >= 0 && ie < SW) sw[c][ie] = (m > L - 1) ? so : se;
-                if (ie + 1 >= 0 && ie + 1 < SW) sw[c][ie + 1] = (m < 0) ? se : so;
-            }
+            const float se = fmaf(sin_sq_fast(al, ue), ib, ue);
+            const float so = fmaf(sin_sq_fast(al, uo), ib, uo);
+            const int ie = 2 * m - n_start;
+            if (ie >= 0 && ie < SW) sc[ie] = (m > L - 1) ? so : se;
+            if (ie + 1 >= 0 && ie + 1 < SW) sc[ie + 1] = (m < 0) ? se : so;
         }
     }
     __syncthreads();
-    // decimate, zero outside [0, L), split into head and tail: 2 rows x 4 channels per item
-    const int npairs = (rows + 1) >> 1;
-    for (int it = tid; it < 2 * npairs; it += NT_ACT) {
-        const int rp = it >> 1, hf = it & 1;
-        const int q0 = 2 * rp;
-        float a0[4], a1[4];
-        if (any_inside) {
+    // decimate, zero outside [0, L), split into head and tail, one 16-byte row per thread
+    for (int q = tid; q < rows; q += NT_ACT) {
+        const int t = t0 + q;
+        float a[8];
+        if (t >= 0 && t < L) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const float2* sr = reinterpret_cast<const float2*>(&sw[4 * hf + cc][2 * q0]);
-                float s[14];
+            for (int cc = 0; cc < 8; ++cc) {
+                const float2* sr = reinterpret_cast<const float2*>(sw + cc * SG + 2 * q);
+                float v = 0.f;
 #pragma unroll
-                for (int j = 0; j < 7; ++j) {
+                for (int j = 0; j < kFilterTaps / 2; ++j) {
                     const float2 s2 = sr[j];
-                    s[2 * j] = s2.x;
-                    s[2 * j + 1] = s2.y;
+                    v = fmaf(p.filt.down[2 * j], s2.x, v);
+                    v = fmaf(p.filt.down[2 * j + 1], s2.y, v);
                 }
-                float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-                for (int j = 0; j < kFilterTaps; ++j) {
-                    v0 = fmaf(p.filt.down[j], s[j], v0);
-                    v1 = fmaf(p.filt.down[j], s[j + 2], v1);
-                }
-                a0[cc] = v0;
-                a1[cc] = v1;
+                a[cc] = v;
             }
+        } else {
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) a[cc] = 0.f;
         }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int q = q0 + r;
-            if (q >= rows) break;
-            const int t = t0 + q;
-            const bool in = t >= 0 && t < L;
-            float v[4];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) v[cc] = in ? (r == 0 ? a0[cc] : a1[cc]) : 0.f;
-            uint2 hv, lv;
-            split2(v[0], v[1], &hv.x, &lv.x);
-            split2(v[2], v[3], &hv.y, &lv.y);
-            reinterpret_cast<uint2*>(ohi + t)[hf] = hv;
-            reinterpret_cast<uint2*>(olo + t)[hf] = lv;
+        uint4 hv, lv;
+        split2(a[0], a[1], &hv.x, &lv.x);
+        split2(a[2], a[3], &hv.y, &lv.y);
+        split2(a[4], a[5], &hv.z, &lv.z);
+        split2(a[6], a[7], &hv.w, &lv.w);
+        ohi[t] = hv;
+        olo[t] = lv;
+    }
+}
+
+// grid: x = row tiles over [-pad_l, L + pad_r), y = B * C / 8 (item, group), z = job
+__global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
+    __shared__ __align__(16) float buf[SMEM_FLOATS];
+    const ActJob& J = p.job[blockIdx.z];
+    const int L = p.L;
+    const int ngroups = p.C / 8;
+    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
+    const int t0 = -p.pad_l + blockIdx.x * TT;           // first output row of the tile
+    const int rows = min(TT, L + p.pad_r - t0);
+    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
+    uint4* ohi = reinterpret_cast<uint4*>(J.a_hi) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
+    uint4* olo = reinterpret_cast<uint4*>(J.a_lo) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
+    if (t0 >= 8 && t0 + TT + 8 <= L) {
+        act_tile_fast(p, J, buf, b, g, t0, ohi, olo);
+    } else {
+        for (int sub = 0; sub < rows; sub += TG) {
+            act_tile_general(p, J, buf, b, g, t0 + sub, min(TG, rows - sub), ohi, olo);
+            __syncthreads();
         }
     }
 }
