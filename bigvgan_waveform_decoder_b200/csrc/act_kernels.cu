@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 
 #include "act_kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace mh3a {
 namespace {
@@ -109,7 +110,10 @@ __device__ __forceinline__ void act_tile_fast(const ActParams& p, const ActJob& 
     float* xs = buf + c * XF_P;
     float* T = buf + 8 * XF_P;   // [8][TF_P] outputs, skewed
     const float* xrow = J.x + ((long long)b * p.C + g * 8 + c) * p.L + (t0 - 8);
-    for (int i = lane; i < XF; i += 32) xs[skew(i)] = __ldg(xrow + i);
+    // all of the window's loads in flight at once (asynchronous copies straight to shared)
+    for (int i = lane; i < XF; i += 32) ptx::cp_async4(xs + skew(i), xrow + i);
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
     __syncwarp();
     const float al = __ldg(J.alpha + g * 8 + c), ib = __ldg(J.inv_beta + g * 8 + c);
     const int q0 = RUN * lane;
@@ -174,7 +178,9 @@ __device__ __forceinline__ void act_tile_general(const ActParams& p, const ActJo
         const int XW = rows + 12;
         const float* xrow = J.x + ((long long)b * C + g * 8 + c) * L;
         float* xc = xs + c * XG;
-        for (int q = lane; q < XW; q += 32) xc[q] = __ldg(xrow + clampi(xs_start + q, 0, L - 1));
+        for (int q = lane; q < XW; q += 32) ptx::cp_async4(xc + q, xrow + clampi(xs_start + q, 0, L - 1));
+        ptx::cp_async_commit();
+        ptx::cp_async_wait_all();
         __syncwarp();
         // SnakeBeta at the 2x rate over n in [2 t0 - 5, 2 (t0 + rows) + 5): a lane takes one
         // input position m and forms both phases; positions past either end repeat the end.
@@ -255,7 +261,46 @@ __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
     }
 }
 
+// Plain head/tail split (no activation) into the same row layout, of x0 or of the mean
+// (x0 + x1 + x2) / 3 of three block outputs.  grid: x = row tiles of NT_ACT, y = B * C / 8.
+__global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
+    const int L = p.L, ngroups = p.C / 8;
+    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
+    const int t = -p.pad_l + blockIdx.x * NT_ACT + threadIdx.x;
+    if (t >= L + p.pad_r) return;
+    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
+    const long long row = ((long long)b * ngroups + g) * Lpad + p.pad_l + t;
+    float v[8];
+    if (t >= 0 && t < L) {
+        const long long base = ((long long)b * p.C + g * 8) * L + t;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const long long i = base + (long long)c * L;
+            v[c] = p.x1 ? (__ldg(p.x0 + i) + __ldg(p.x1 + i) + __ldg(p.x2 + i)) / 3.0f : __ldg(p.x0 + i);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = 0.f;
+    }
+    uint4 hv, lv;
+    split2(v[0], v[1], &hv.x, &lv.x);
+    split2(v[2], v[3], &hv.y, &lv.y);
+    split2(v[4], v[5], &hv.z, &lv.z);
+    split2(v[6], v[7], &hv.w, &lv.w);
+    reinterpret_cast<uint4*>(p.a_hi)[row] = hv;
+    reinterpret_cast<uint4*>(p.a_lo)[row] = lv;
+}
+
 }  // namespace
+
+int launch_split_rows(const SplitParams& p, cudaStream_t s) {
+    if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0 || !p.x0) return -1;
+    if ((p.x1 == nullptr) != (p.x2 == nullptr)) return -1;
+    const int total = p.L + p.pad_l + p.pad_r;
+    dim3 grid((total + NT_ACT - 1) / NT_ACT, p.B * (p.C / 8));
+    k_split_rows<<<grid, NT_ACT, 0, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
 
 int launch_act_split(const ActParams& p, int njobs, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0) return -1;

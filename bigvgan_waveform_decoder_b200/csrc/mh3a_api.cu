@@ -41,7 +41,7 @@ constexpr int kMaxSegments = 2 + 2 * MH3A_MAX_STAGES + 1;
 // sequence at least the largest conv padding, after it the largest tile overhang (2 x 128
 // rows) plus that padding.
 constexpr int kApadL = 32;
-constexpr int kApadR = 2 * 128 + 32;
+constexpr int kApadR = 4 * 128 + 32;
 
 // Kaiser-windowed sinc low-pass of the activation (FastVideo "minimax_h3_audio_vae" page,
 // `kaiser_sinc_filter1d`): Kaiser's estimate A = 2.285 (K/2 - 1) pi (4 hw) + 7.95 of the stop-band

@@ -733,6 +733,334 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
 }
 
 // ----------------------------------------------------------------------------------------------
+// persistent AMP GEMM: one CTA per SM walks a list of output tiles (job, item, 128 MT time rows,
+// NT output channels).  The tile's K loop is cut into passes of at most 8 MMA K-steps; each
+// pass accumulates head x head and both cross products into one of two TMEM buffers, and the
+// epilogue warps fold the finished buffer into fp32 registers (round to nearest) while the
+// tensor core fills the other.  A pass therefore holds at most 24 truncating accumulations,
+// the epilogue of one tile overlaps the MMAs of the next, and A / B stream through rings of
+// bulk copies that run several stages ahead.
+// ----------------------------------------------------------------------------------------------
+// EW epilogue warps (EW / 4 per TMEM lane quarter) after warp 0 (MMA) and warp 1 (loader).
+constexpr int ps_threads(int EW) { return 64 + 32 * EW; }
+constexpr int PS_MAXS = 8;                              // ring stages (max)
+constexpr int PS_BUFCOLS = 256;                         // TMEM columns per accumulator buffer
+
+struct PsPlan {
+    int RS;             // window rows per channel group (max over jobs)
+    int SA, SB;         // bytes per A / B ring stage
+    int nsa, nsb;       // ring depths
+    int offB, offBar;
+    int smem;
+};
+
+struct PsSched {
+    int ntiles, n_ot, per_job;   // tiles in all, output-channel tiles, tiles per job
+    int pu;                      // tap units per pass
+};
+
+// Tile k of the launch (jobs sorted by cost, heaviest first).
+struct PsTile {
+    int z, b, t0, ot;
+};
+
+template <int MT>
+__device__ __forceinline__ PsTile ps_tile(const GemmParams& p, const PsSched& sc, int k) {
+    PsTile T;
+    T.z = k / sc.per_job;
+    int r = k - T.z * sc.per_job;
+    const int per_b = p.tiles_t * sc.n_ot;
+    T.b = r / per_b;
+    r -= T.b * per_b;
+    const int tt = r / sc.n_ot;
+    T.ot = r - tt * sc.n_ot;
+    T.t0 = tt * 128 * MT;
+    return T;
+}
+
+// The i-th tile of this CTA: rounds of gridDim.x tiles, walked forwards and backwards in turn
+// so that a CTA that drew a heavy tile in one round draws a light one in the next.
+__device__ __forceinline__ int ps_tile_index(int i, int ntiles) {
+    const int G = gridDim.x;
+    const int base = i * G;
+    if (base >= ntiles) return -1;
+    const int k = base + ((i & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+    return k < ntiles ? k : -1;
+}
+
+template <int MT, int NT, int KGT, int EW>
+__global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    static_assert(MT * NT <= PS_BUFCOLS, "one accumulator buffer holds MT x NT columns");
+    static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
+    static_assert(EW == 8 || EW == 16, "epilogue warps");
+    static_assert((4 * MT * NT / EW) % 16 == 0 && 4 * MT * NT / EW <= NT, "epilogue column split");
+    constexpr int BG = (KGT == 1) ? 2 : KGT;
+    constexpr int TAPB = 2 * BG * NT * 16;
+    constexpr int CW = 4 * MT * NT / EW;                // accumulator columns per epilogue warp
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Cin = p.Cin, Cout = p.Cout, L = p.L;
+    const int nchunks = Cin / (8 * KGT);
+    const int TPU = p.tpu, PU = sc.pu;
+    const int RS = pl.RS, nsa = pl.nsa, nsb = pl.nsb;
+
+    uint8_t* As = smem;
+    uint8_t* Bs = smem + pl.offB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
+    uint64_t* a_full = bars;
+    uint64_t* a_empty = bars + PS_MAXS;
+    uint64_t* b_full = bars + 2 * PS_MAXS;
+    uint64_t* b_empty = bars + 3 * PS_MAXS;
+    uint64_t* acc_full = bars + 4 * PS_MAXS;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* done_bar = acc_full + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nsa; ++s) {
+            ptx::mbar_init(&a_full[s], 1);
+            ptx::mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < nsb; ++s) {
+            ptx::mbar_init(&b_full[s], 1);
+            ptx::mbar_init(&b_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&acc_full[s], 1);
+            ptx::mbar_init(&acc_empty[s], EW);
+        }
+        ptx::mbar_init(done_bar, 1);
+        *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, 2 * PS_BUFCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            // Descriptors are built once per ring slot and then advanced by adding 16-byte
+            // offsets to their low word (the start-address field), so that issuing an MMA costs
+            // a few integer adds: narrow tiles finish an MMA in 16 cycles.
+            constexpr uint32_t idesc = ptx::idesc_bf16(128, NT);
+            constexpr int KK = (KGT == 1) ? 1 : KGT / 2;   // K-steps per tap unit
+            const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
+            bool ok = *abort_flag == 0;
+            int sa = 0, sb = 0, buf = 0;
+            uint32_t pa = 0, pb = 0, pacc = 0;   // phase bits of the slots in use
+            for (int i = 0; ok; ++i) {
+                const int k = ps_tile_index(i, sc.ntiles);
+                if (k < 0) break;
+                const PsTile T = ps_tile<MT>(p, sc, k);
+                const GemmJob& J = p.job[T.z];
+                const int K = J.K, dil = J.dil;
+                const int KU = (KGT == 1) ? (K + 1) / 2 : K;
+                const uint32_t step = (uint32_t)((KGT == 1 ? 2 : 1) * dil);   // window rows per unit
+                const uint32_t a_lbo = (KGT == 1) ? (uint32_t)dil * 16 : (uint32_t)RS * 16;
+                for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
+                    if (!ptx::mbar_wait(&a_full[sa], pa, kWaitLimit)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t ah0 = ptx::desc_lo(a_smem + sa * pl.SA, a_lbo);
+                    int ucopy = 0, upass = 0;
+                    uint32_t bh0 = 0, ashift = 0;
+                    for (int unit = 0; unit < KU; ++unit, ashift += step) {
+                        if (ucopy == 0) {
+                            if (!ptx::mbar_wait(&b_full[sb], pb, kWaitLimit)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            bh0 = ptx::desc_lo(b_smem + sb * pl.SB, NT * 16);
+                        }
+                        if (upass == 0) {
+                            if (!ptx::mbar_wait(&acc_empty[buf], pacc ^ 1, kWaitLimit)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                        }
+                        // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
+                        // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
+                        const uint32_t bh = bh0 + (uint32_t)ucopy * (TAPB >> 4);
+                        const uint32_t dbase = tmem + (uint32_t)(buf * PS_BUFCOLS);
+#pragma unroll
+                        for (int kk = 0; kk < KK; ++kk) {
+                            const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
+                            const uint32_t blk = bhk + (uint32_t)(BG * NT);
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt) {
+                                const uint32_t a = ah0 + ashift + (uint32_t)(2 * kk * RS + mt * 128);
+                                const uint32_t d = dbase + (uint32_t)(mt * NT);
+                                ptx::mma_bf16(d, ptx::desc64(a), ptx::desc64(bhk), idesc, (upass == 0 && kk == 0) ? 0u : 1u);
+                                ptx::mma_bf16(d, ptx::desc64(a), ptx::desc64(blk), idesc, 1u);
+                                ptx::mma_bf16(d, ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bhk), idesc, 1u);
+                            }
+                        }
+                        ++ucopy;
+                        ++upass;
+                        if (ucopy == TPU || unit == KU - 1) {
+                            ptx::mma_commit(&b_empty[sb]);
+                            ucopy = 0;
+                            if (++sb == nsb) { sb = 0; pb ^= 1; }
+                        }
+                        if (upass == PU || unit == KU - 1) {
+                            ptx::mma_commit(&acc_full[buf]);
+                            upass = 0;
+                            buf ^= 1;
+                            if (buf == 0) pacc ^= 1;
+                        }
+                    }
+                    if (!ok) break;
+                    ptx::mma_commit(&a_empty[sa]);
+                    if (++sa == nsa) { sa = 0; pa ^= 1; }
+                    if (*abort_flag) ok = false;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(p.err, 5);
+            }
+            // every MMA issued has completed before the CTA releases its tensor memory
+            ptx::mma_commit(done_bar);
+            ptx::mbar_wait(done_bar, 0, kWaitLimit);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- A and B loader
+        if (lane == 0) {
+            const size_t unit_elems = (size_t)2 * BG * NT * 8;
+            bool ok = *abort_flag == 0;
+            int ia = 0, ib = 0;
+            for (int i = 0; ok; ++i) {
+                const int k = ps_tile_index(i, sc.ntiles);
+                if (k < 0) break;
+                const PsTile T = ps_tile<MT>(p, sc, k);
+                const GemmJob& J = p.job[T.z];
+                const int K = J.K, dil = J.dil;
+                const int KU = (KGT == 1) ? (K + 1) / 2 : K;
+                const int NUC = (KU + TPU - 1) / TPU;
+                const int ROWS = 128 * MT + (K - 1) * dil + (KGT == 1 ? dil : 0);
+                const uint32_t a_bytes = (uint32_t)(2 * KGT * ROWS * 16);
+                const long long row0 = p.pad_l + T.t0 - J.pad;   // first window row in the A arrays
+                const uint16_t* wsrc = J.w + (size_t)T.ot * nchunks * KU * unit_elems;
+                for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
+                    const int sa = ia % nsa;
+                    if (!ptx::mbar_wait(&a_empty[sa], ((ia / nsa) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&a_full[sa], a_bytes);
+                    for (int part = 0; part < 2; ++part) {
+                        const uint8_t* base = part == 0 ? J.a_hi : J.a_lo;
+                        for (int g = 0; g < KGT; ++g) {
+                            const long long grp = (long long)T.b * (Cin / 8) + chunk * KGT + g;
+                            ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KGT + g) * RS) * 16,
+                                          base + (grp * p.Lpad + row0) * 16, (uint32_t)(ROWS * 16), &a_full[sa]);
+                        }
+                    }
+                    ++ia;
+                    for (int uc = 0; uc < NUC; ++uc) {
+                        const int sb = ib % nsb;
+                        if (!ptx::mbar_wait(&b_empty[sb], ((ib / nsb) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                        // tap units [uc * TPU, min(KU, (uc + 1) * TPU)) are contiguous in the packing
+                        const int nunits = min(KU, (uc + 1) * TPU) - uc * TPU;
+                        const uint32_t bytes = (uint32_t)(nunits * TAPB);
+                        ptx::mbar_arrive_expect_tx(&b_full[sb], bytes);
+                        ptx::bulk_g2s(Bs + (size_t)sb * pl.SB,
+                                      wsrc + ((size_t)chunk * KU + (size_t)uc * TPU) * unit_elems, bytes, &b_full[sb]);
+                        ++ib;
+                    }
+                    if (*abort_flag) ok = false;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(p.err, 6);
+            }
+            // let the copies still in flight land before the CTA can exit
+            for (int c = (ia > nsa ? ia - nsa : 0); c < ia; ++c)
+                ptx::mbar_wait(&a_full[c % nsa], (c / nsa) & 1, kWaitLimit);
+            for (int v = (ib > nsb ? ib - nsb : 0); v < ib; ++v)
+                ptx::mbar_wait(&b_full[v % nsb], (v / nsb) & 1, kWaitLimit);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2 .. EW+1)
+        const int e = warp - 2;
+        const int q4 = warp & 3;               // TMEM lane quarter this warp may access
+        const int col0 = (e >> 2) * CW;        // first accumulator column of this warp
+        const int mt = col0 / NT, oc0 = col0 % NT;
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)col0;
+        constexpr bool kPrefetch = CW <= 16;   // residual loaded ahead while the MMAs run
+        bool ok = *abort_flag == 0;
+        int ip = 0;
+        for (int i = 0; ok; ++i) {
+            const int k = ps_tile_index(i, sc.ntiles);
+            if (k < 0) break;
+            const PsTile T = ps_tile<MT>(p, sc, k);
+            const GemmJob& J = p.job[T.z];
+            const int KU = (KGT == 1) ? (J.K + 1) / 2 : J.K;
+            const int npass = nchunks * ((KU + PU - 1) / PU);
+            const int t = T.t0 + mt * 128 + q4 * 32 + lane;
+            const int o_base = T.ot * NT + oc0;
+            const long long idx0 = ((long long)T.b * Cout + o_base) * L + t;
+            float res[kPrefetch ? CW : 1];
+            if (kPrefetch) {
+#pragma unroll
+                for (int c = 0; c < CW; ++c)
+                    res[c] = (J.res && t < L && o_base + c < Cout) ? J.res[idx0 + (long long)c * L] : 0.f;
+            }
+            float acc[CW];
+#pragma unroll
+            for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+            for (int ps = 0; ps < npass; ++ps, ++ip) {
+                const int buf = ip & 1;
+                if (!ptx::mbar_wait(&acc_full[buf], (ip >> 1) & 1, kWaitLimit)) { ok = false; break; }
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int cb = 0; cb < CW; cb += 16) {
+                    float v[16];
+                    ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + cb), v);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) acc[cb + c] += v[c];
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+            }
+            if (!ok || *abort_flag) {
+                ok = false;
+                break;
+            }
+            if (t < L) {
+                // FC columns at a time: all loads of a group are in flight before its stores
+                constexpr int FC = (CW > 64) ? 8 : 16;
+#pragma unroll
+                for (int cb = 0; cb < CW; cb += FC) {
+                    float bs[FC], rs[FC];
+#pragma unroll
+                    for (int c = 0; c < FC; ++c) {
+                        const int o = o_base + cb + c;   // channels past Cout pad the tile
+                        bs[c] = (o < Cout) ? __ldg(J.bias + o) : 0.f;
+                        if (kPrefetch) rs[c] = res[cb + c];
+                        else rs[c] = (J.res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * L] : 0.f;
+                    }
+#pragma unroll
+                    for (int c = 0; c < FC; ++c)
+                        if (o_base + cb + c < Cout) J.out[idx0 + (long long)(cb + c) * L] = (acc[cb + c] + bs[c]) + rs[c];
+                }
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            atomicExch(p.err, 7);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 0) ptx::tmem_dealloc(tmem, 2 * PS_BUFCOLS);
+}
+
+// ----------------------------------------------------------------------------------------------
 // host side
 // ----------------------------------------------------------------------------------------------
 
@@ -751,7 +1079,7 @@ float bf16_value(uint16_t h) {
 }
 
 // Output-channel tile of each layer kind (the weight blocks are laid out for it).
-int ntile_amp(int C) { return C >= 64 ? 64 : C; }
+int ntile_amp(int C) { return C >= 128 ? 128 : (C >= 64 ? 64 : C); }
 int ntile_pre(int) { return 64; }
 int ntile_convt(int Cout, int r) {
     if (r > 2) return Cout >= 32 ? 32 : Cout;
@@ -813,9 +1141,9 @@ int launch_tc(const TcParams& p0, int njobs, cudaStream_t s) {
 // bias of these stages dominated the decode error with a single head accumulator).
 int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
-        case 256: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
-        case 128: return launch_tc<MODE_AMP, 1, 64, 4, 1>(p, njobs, s);
+        case 512: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
+        case 256: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
+        case 128: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
         case 64: return launch_tc<MODE_AMP, 2, 64, 3, 1>(p, njobs, s);
         case 32: return launch_tc<MODE_AMP, 2, 32, 2, 1>(p, njobs, s);
         default: return -1;
@@ -862,15 +1190,77 @@ int launch_gemm(const GemmParams& p0, int njobs, cudaStream_t s) {
 }
 
 // GEMM tile shape per width; NT and the channels per chunk must match amp_layout().
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <int MT, int NT, int KGT, int EW>
+int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
+    GemmParams p = p0;
+    const int kc = 8 * KGT;
+    if (p.Cin % kc != 0 || njobs < 1) return -1;
+    p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
+    int span = 0, padmax = 0, dilmax = 0, kumax = 1;
+    for (int j = 0; j < njobs; ++j) {
+        span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
+        padmax = std::max(padmax, p.job[j].pad);
+        dilmax = std::max(dilmax, p.job[j].dil);
+        kumax = std::max(kumax, KGT == 1 ? (p.job[j].K + 1) / 2 : p.job[j].K);
+    }
+    const int extra = (KGT == 1) ? dilmax : 0;   // the phantom tap of the last tap pair
+    // every window row the tiles touch must exist in the A arrays
+    if (p.pad_l < padmax ||
+        p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax + extra)
+        return -1;
+    constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * NT * 16;
+    p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));   // weight copies of about 16 KB
+    PsSched sc{};
+    sc.n_ot = (p.Cout + NT - 1) / NT;
+    sc.per_job = p.B * p.tiles_t * sc.n_ot;
+    sc.ntiles = njobs * sc.per_job;
+    sc.pu = (KGT == 4) ? 4 : 8;                             // 8 MMA K-steps per pass
+    PsPlan pl{};
+    pl.RS = 128 * MT + span + extra;
+    pl.SA = 2 * KGT * pl.RS * 16;
+    pl.SB = p.tpu * TAPB;
+    constexpr int kBudget = 227 * 1024 - (8 * (4 * PS_MAXS + 5) + 16) - 64;
+    pl.nsa = (4 * pl.SA <= kBudget / 2) ? 4 : 3;
+    if (pl.nsa * pl.SA + 2 * pl.SB > kBudget) pl.nsa = 2;
+    pl.nsb = std::min(PS_MAXS, (kBudget - pl.nsa * pl.SA) / pl.SB);
+    if (pl.nsb < 2) return -1;
+    pl.offB = pl.nsa * pl.SA;
+    pl.offBar = (pl.offB + pl.nsb * pl.SB + 15) / 16 * 16;
+    pl.smem = pl.offBar + 8 * (4 * PS_MAXS + 5) + 16;
+    // at least half the SM's shared memory, so that a second CTA never waits on the first's
+    // tensor memory
+    const int smem_req = std::max(pl.smem, 116 * 1024);
+    if (smem_req > 227 * 1024) return -1;
+    const int nsm = sm_count();
+    if (nsm <= 0) return -1;
+    auto kern = k_gemm_ps<MT, NT, KGT, EW>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_req) != cudaSuccess) return -1;
+    const int grid = std::min(sc.ntiles, nsm);
+    kern<<<grid, ps_threads(EW), smem_req, s>>>(p, sc, pl);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
+
 int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
-        case 256: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
-        case 128: return launch_gemm<1, 64, 4, 4>(p, njobs, s);
-        case 64: return launch_gemm<1, 64, 3, 4>(p, njobs, s);
-        case 32: return launch_gemm<2, 32, 2, 4>(p, njobs, s);
-        case 16: return launch_gemm<2, 16, 2, 2>(p, njobs, s);
-        case 8: return launch_gemm<2, 16, 2, 1>(p, njobs, s);
+        case 512: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
+        case 256: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
+        case 128: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
+        case 64: return launch_gemm_ps<2, 64, 4, 16>(p, njobs, s);
+        case 32: return launch_gemm_ps<2, 32, 4, 16>(p, njobs, s);
+        case 16: return launch_gemm_ps<4, 16, 2, 16>(p, njobs, s);
+        case 8: return launch_gemm_ps<4, 16, 1, 16>(p, njobs, s);
         default: return -1;
     }
 }

@@ -162,6 +162,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// The same descriptor split into words: the low word holds the start address and `lbo`, the
+// high word `sbo` = 128 bytes and the version bit.  Adding n to the low word moves the start
+// address by 16 n bytes (shared addresses stay below 2^18, so the 14-bit field never carries).
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc64(uint32_t lo) {
+    constexpr uint32_t hi = (128u >> 4) | (1u << 14);
+    return ((uint64_t)hi << 32) | lo;
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B (K-major), fp32 D, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
     return (1u << 4)                          // D format: f32
