@@ -14,11 +14,12 @@
 // are written as zeros: they are the conv's zero padding, so the GEMM never special-cases the
 // sequence ends.  Heads and tails go to separate arrays.
 //
-// A block covers TT = 512 output rows of one channel group.  Tiles away from the sequence ends
-// take the fast path: every lane owns 16 consecutive outputs of one channel, forms the 32
-// SnakeBeta values at the 2x rate that belong to them in registers, receives the 5 + 5 halo
-// values from its neighbour lanes by warp shuffles, and decimates in registers.  The tiles at
-// the ends take the general path, which clamps every index.
+// A block covers TT = 512 output rows of one channel group.  Every lane owns 16 consecutive
+// outputs of one channel, forms the 32 SnakeBeta values at the 2x rate that belong to them in
+// registers, receives the 5 + 5 halo values from its neighbour lanes by warp shuffles, and
+// decimates in registers; a shared-memory transpose then packs rows of 8 channels.  Tiles that
+// touch a sequence end clamp the input index and substitute the end values at the 2x rate
+// (the replicate paddings); tiles wholly outside the sequence only write zero rows.
 #include <cuda_bf16.h>
 
 #include "act_kernels.cuh"
@@ -28,19 +29,15 @@ namespace mh3a {
 namespace {
 
 constexpr int TT = 512;                   // output rows per block
-constexpr int RUN = 16;                   // outputs per lane on the fast path (TT = 32 RUN)
-constexpr int TG = 256;                   // rows per sub-tile of the general path
+constexpr int RUN = 16;                   // outputs per lane (TT = 32 RUN)
 constexpr int NT_ACT = 256;               // threads per block (8 warps: one per channel)
 constexpr int NS = 2 * RUN + 10;          // SnakeBeta values one lane's decimation reads
-// Fast-path shared layout: per channel a window of x and a row of outputs, each with 4 floats
+// Shared layout: per channel a window of x and a row of outputs, each with 4 floats
 // of padding after every 16 so that lanes reading 16-float runs hit distinct banks.
 constexpr int XF = TT + 16;               // x[t0 - 8, t0 + TT + 8)
 constexpr int XF_P = XF + XF / 16 * 4;
 constexpr int TF_P = TT + TT / 16 * 4;
-// General-path shared layout.
-constexpr int XG = TG + 16;
-constexpr int SG = 2 * TG + 12;
-constexpr int SMEM_FLOATS = (8 * (XF_P + TF_P) > 8 * (XG + SG)) ? 8 * (XF_P + TF_P) : 8 * (XG + SG);
+constexpr int SMEM_FLOATS = 8 * (XF_P + TF_P);
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 __device__ __forceinline__ int skew(int i) { return i + ((i >> 4) << 2); }
@@ -76,10 +73,6 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t* h, uint32_t* 
     *l = pack2(a - ha, b - hb);
 }
 
-// ---------------------------------------------------------------------------------------------
-// fast path: rows [t0, t0 + TT) with 8 <= t0 and t0 + TT + 8 <= L, so that neither the input
-// window nor the 2x-rate SnakeBeta window reaches past a sequence end
-// ---------------------------------------------------------------------------------------------
 
 // SnakeBeta value j of a lane's window, n = 2 (t0 + q0) - 5 + j, from xv[k] = x[t0 + q0 - 8 + k]
 // (j even: odd phase n = 2m + 1; j odd: even phase n = 2m).
@@ -104,14 +97,33 @@ __device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv,
     }
 }
 
-__device__ __forceinline__ void act_tile_fast(const ActParams& p, const ActJob& J, float* buf, int b,
-                                              int g, int t0, uint4* ohi, uint4* olo) {
+// One tile: rows [t0, t0 + TT).  EDGE = false requires 8 <= t0 and t0 + TT + 8 <= L, so that
+// neither the input window nor the 2x-rate SnakeBeta window reaches past a sequence end.  EDGE
+// tiles clamp the input index (the replicate padding of x), replace SnakeBeta values outside
+// [0, 2L) by the end values (the replicate padding at the 2x rate), and write zero rows
+// outside [0, L).
+template <bool EDGE>
+__device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, float* buf, int b, int g, int t0,
+                                         int rows, uint4* ohi, uint4* olo) {
+    const int L = p.L;
     const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
     float* xs = buf + c * XF_P;
     float* T = buf + 8 * XF_P;   // [8][TF_P] outputs, skewed
-    const float* xrow = J.x + ((long long)b * p.C + g * 8 + c) * p.L + (t0 - 8);
-    // all of the window's loads in flight at once (asynchronous copies straight to shared)
-    for (int i = lane; i < XF; i += 32) ptx::cp_async4(xs + skew(i), xrow + i);
+    const float* xrow = J.x + ((long long)b * p.C + g * 8 + c) * L;
+    // all of the window's loads in flight at once (asynchronous copies straight to shared);
+    // skew(lane + 32 k) = skew(lane) + 40 k
+    {
+        float* dst = xs + skew(lane);
+#pragma unroll
+        for (int k = 0; k < (XF + 31) / 32; ++k) {
+            const int i = lane + 32 * k;
+            if (i < XF) {
+                int src = t0 - 8 + i;
+                if (EDGE) src = clampi(src, 0, L - 1);
+                ptx::cp_async4(dst + 40 * k, xrow + src);
+            }
+        }
+    }
     ptx::cp_async_commit();
     ptx::cp_async_wait_all();
     __syncwarp();
@@ -128,13 +140,39 @@ __device__ __forceinline__ void act_tile_fast(const ActParams& p, const ActJob& 
     }
     float s[NS];
     snake_range<5, 5 + 2 * RUN>(p.filt, xv, al, ib, s);     // the lane's own 2 RUN values
+    // The 5 values left of lane 0's run and right of lane 31's run: lanes 0-4 and 5-9 form one
+    // each (value j of lane 0's window, resp. j = 37 .. 41 of lane 31's), from the same taps.
+    float hv = 0.f;
+    if (lane < 10) {
+        const int j = (lane < 5) ? lane : lane + 2 * RUN;
+        const int i0 = ((lane < 5) ? 0 : RUN * 31) + 8 + (j >> 1);
+        const int par = j & 1;
+        float u = 0.f;
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k + par], xs[skew(i0 - k)], u);
+        hv = fmaf(sin_sq_fast(al, u), ib, u);
+    }
 #pragma unroll
     for (int j = 0; j < 5; ++j) {
-        s[j] = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
-        s[j + 5 + 2 * RUN] = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
+        const float from_left = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
+        const float from_right = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
+        const float h = __shfl_sync(0xffffffffu, hv, (lane == 31) ? j + 5 : j);
+        s[j] = (lane == 0) ? h : from_left;
+        s[j + 5 + 2 * RUN] = (lane == 31) ? h : from_right;
     }
-    if (lane == 0) snake_range<0, 5>(p.filt, xv, al, ib, s);
-    if (lane == 31) snake_range<5 + 2 * RUN, NS>(p.filt, xv, al, ib, s);
+    if (EDGE) {
+        // replicate padding at the 2x rate: n < 0 takes s(0), n > 2L - 1 takes s(2L - 1)
+        const int n0 = 2 * (t0 + q0) - 5;
+        const int j0 = -n0, je = 2 * L - 1 - n0;
+        float sf = s[0], sl = s[NS - 1];
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            sf = (j == j0) ? s[j] : sf;
+            sl = (j == je) ? s[j] : sl;
+        }
+#pragma unroll
+        for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
+    }
     float a[RUN];
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
@@ -148,94 +186,27 @@ __device__ __forceinline__ void act_tile_fast(const ActParams& p, const ActJob& 
     for (int k = 0; k < RUN / 4; ++k)
         *reinterpret_cast<float4*>(trow + skew(q0 + 4 * k)) = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
     __syncthreads();
-    for (int q = tid; q < TT; q += NT_ACT) {
-        const int qs = skew(q);
+    // rows of 8 channels: skew(q + 256) = skew(q) + 320
+#pragma unroll
+    for (int r = 0; r < TT / NT_ACT; ++r) {
+        const int q = tid + r * NT_ACT;
+        if (EDGE && q >= rows) break;
+        const int qs = skew(tid) + r * (NT_ACT + NT_ACT / 4);
+        const int t = t0 + q;
         float v[8];
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) v[cc] = T[cc * TF_P + qs];
-        uint4 hv, lv;
-        split2(v[0], v[1], &hv.x, &lv.x);
-        split2(v[2], v[3], &hv.y, &lv.y);
-        split2(v[4], v[5], &hv.z, &lv.z);
-        split2(v[6], v[7], &hv.w, &lv.w);
-        ohi[t0 + q] = hv;
-        olo[t0 + q] = lv;
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
-// general path: rows [t0, t0 + rows), rows <= TG, anywhere in [-pad_l, L + pad_r)
-// ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void act_tile_general(const ActParams& p, const ActJob& J, float* buf, int b,
-                                                 int g, int t0, int rows, uint4* ohi, uint4* olo) {
-    const int C = p.C, L = p.L;
-    const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
-    float* xs = buf;              // [8][XG]
-    float* sw = buf + 8 * XG;     // [8][SG]
-    const bool any_inside = t0 < L && t0 + rows > 0;
-    if (any_inside) {
-        const int xs_start = t0 - 6;
-        const int XW = rows + 12;
-        const float* xrow = J.x + ((long long)b * C + g * 8 + c) * L;
-        float* xc = xs + c * XG;
-        for (int q = lane; q < XW; q += 32) ptx::cp_async4(xc + q, xrow + clampi(xs_start + q, 0, L - 1));
-        ptx::cp_async_commit();
-        ptx::cp_async_wait_all();
-        __syncwarp();
-        // SnakeBeta at the 2x rate over n in [2 t0 - 5, 2 (t0 + rows) + 5): a lane takes one
-        // input position m and forms both phases; positions past either end repeat the end.
-        const float al = __ldg(J.alpha + g * 8 + c), ib = __ldg(J.inv_beta + g * 8 + c);
-        const int n_start = 2 * t0 - 5, SW = 2 * rows + 10;
-        const float* xr0 = xc - xs_start;
-        float* sc = sw + c * SG;
-        const int m_lo = n_start >> 1, m_hi = (n_start + SW - 1) >> 1;
-        for (int m = m_lo + lane; m <= m_hi; m += 32) {
-            const int mc = clampi(m, 0, L - 1);
-            float xv[7];
+        if (EDGE && (t < 0 || t >= L)) {
 #pragma unroll
-            for (int k = 0; k < 7; ++k) xv[k] = xr0[mc + k - 3];
-            float ue = 0.f, uo = 0.f;
-#pragma unroll
-            for (int k = 0; k < 6; ++k) {
-                ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
-                uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
-            }
-            const float se = fmaf(sin_sq_fast(al, ue), ib, ue);
-            const float so = fmaf(sin_sq_fast(al, uo), ib, uo);
-            const int ie = 2 * m - n_start;
-            if (ie >= 0 && ie < SW) sc[ie] = (m > L - 1) ? so : se;
-            if (ie + 1 >= 0 && ie + 1 < SW) sc[ie + 1] = (m < 0) ? se : so;
+            for (int cc = 0; cc < 8; ++cc) v[cc] = 0.f;
         }
-    }
-    __syncthreads();
-    // decimate, zero outside [0, L), split into head and tail, one 16-byte row per thread
-    for (int q = tid; q < rows; q += NT_ACT) {
-        const int t = t0 + q;
-        float a[8];
-        if (t >= 0 && t < L) {
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const float2* sr = reinterpret_cast<const float2*>(sw + cc * SG + 2 * q);
-                float v = 0.f;
-#pragma unroll
-                for (int j = 0; j < kFilterTaps / 2; ++j) {
-                    const float2 s2 = sr[j];
-                    v = fmaf(p.filt.down[2 * j], s2.x, v);
-                    v = fmaf(p.filt.down[2 * j + 1], s2.y, v);
-                }
-                a[cc] = v;
-            }
-        } else {
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) a[cc] = 0.f;
-        }
-        uint4 hv, lv;
-        split2(a[0], a[1], &hv.x, &lv.x);
-        split2(a[2], a[3], &hv.y, &lv.y);
-        split2(a[4], a[5], &hv.z, &lv.z);
-        split2(a[6], a[7], &hv.w, &lv.w);
-        ohi[t] = hv;
-        olo[t] = lv;
+        uint4 hv4, lv4;
+        split2(v[0], v[1], &hv4.x, &lv4.x);
+        split2(v[2], v[3], &hv4.y, &lv4.y);
+        split2(v[4], v[5], &hv4.z, &lv4.z);
+        split2(v[6], v[7], &hv4.w, &lv4.w);
+        ohi[t] = hv4;
+        olo[t] = lv4;
     }
 }
 
@@ -252,11 +223,15 @@ __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
     uint4* ohi = reinterpret_cast<uint4*>(J.a_hi) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
     uint4* olo = reinterpret_cast<uint4*>(J.a_lo) + ((long long)b * ngroups + g) * Lpad + p.pad_l;
     if (t0 >= 8 && t0 + TT + 8 <= L) {
-        act_tile_fast(p, J, buf, b, g, t0, ohi, olo);
+        act_tile<false>(p, J, buf, b, g, t0, TT, ohi, olo);
+    } else if (t0 < L && t0 + rows > 0) {
+        act_tile<true>(p, J, buf, b, g, t0, rows, ohi, olo);
     } else {
-        for (int sub = 0; sub < rows; sub += TG) {
-            act_tile_general(p, J, buf, b, g, t0 + sub, min(TG, rows - sub), ohi, olo);
-            __syncthreads();
+        // rows entirely outside [0, L): zeros (the conv's padding)
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        for (int q = threadIdx.x; q < rows; q += NT_ACT) {
+            ohi[t0 + q] = z;
+            olo[t0 + q] = z;
         }
     }
 }

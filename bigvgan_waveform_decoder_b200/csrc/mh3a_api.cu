@@ -349,6 +349,27 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
     return MH3A_OK;
 }
 
+// Head/tail rows of x0 (or of the mean of x0, x1, x2) into the first A operand pair.
+mh3a_status split_to_a(mh3a_handle* h, const float* x0, const float* x1, const float* x2, int C, int L, int B,
+                       cudaStream_t s) {
+    if ((long long)B * C * ((long long)L + kApadL + kApadR) > h->a_cap) {
+        g_last_error = "batch too large for the tensor-core operand buffers (B > max_batch)";
+        return MH3A_ERR_SHAPE;
+    }
+    SplitParams sp{};
+    sp.x0 = x0;
+    sp.x1 = x1;
+    sp.x2 = x2;
+    sp.a_hi = h->A_hi[0];
+    sp.a_lo = h->A_lo[0];
+    sp.C = C;
+    sp.L = L;
+    sp.B = B;
+    sp.pad_l = kApadL;
+    sp.pad_r = kApadR;
+    return counted(h, launch_split_rows(sp, s));
+}
+
 mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* out, cudaStream_t s) {
     const mh3a_config& c = h->cfg;
     h->nseg = 0;
@@ -368,7 +389,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = 1;
         p.job[0].dil = 1;
         p.job[0].pad = 0;
-        if ((st = counted(h, launch_conv_simt(p, 1, false, false, s)))) return st;
+        if ((st = counted(h, launch_conv1x1(p, s)))) return st;
         if ((st = record(h, s))) return st;
     }
     // conv_pre
@@ -385,7 +406,15 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = h->pre.k;
         p.job[0].dil = 1;
         p.job[0].pad = 3;
-        int n = h->pre_tc ? launch_conv_pre_tc(p, h->tc[0], s, h->dev_err) : launch_conv_simt(p, 1, false, false, s);
+        int n;
+        if (h->pre_tc) {
+            // split the input into head/tail rows once, then the persistent tensor-core GEMM
+            if ((st = split_to_a(h, h->buf_in, nullptr, nullptr, c.latent_dim, N, B, s))) return st;
+            n = launch_conv_pre_gemm(p, h->tc[0], h->A_hi[0], h->A_lo[0], kApadL, (long long)N + kApadL + kApadR,
+                                     s, h->dev_err);
+        } else {
+            n = launch_conv_simt(p, 1, false, false, s);
+        }
         if ((st = counted(h, n))) return st;
         if ((st = record(h, s))) return st;
     }
@@ -410,7 +439,14 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             // the fused mean reads exactly three block outputs; otherwise reduce explicitly
             return MH3A_ERR_UNSUPPORTED;
         }
-        const int nl = h->ups_tc[i] ? launch_convT_tc(q, h->tc[i], s, h->dev_err) : launch_convT_simt(q, mean3, s);
+        int nl;
+        if (h->ups_tc[i]) {
+            if ((st = split_to_a(h, q.x0, q.x1, q.x2, C, L, B, s))) return st;
+            nl = launch_convT_gemm(q, h->tc[i], h->A_hi[0], h->A_lo[0], kApadL, (long long)L + kApadL + kApadR, s,
+                                   h->dev_err);
+        } else {
+            nl = launch_convT_simt(q, mean3, s);
+        }
         if ((st = counted(h, nl))) return st;
         if ((st = record(h, s))) return st;
         C /= 2;
@@ -694,11 +730,21 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     const long long n_in = rnd((long long)c.latent_dim * BN), n_pre = rnd((long long)c.decoder_dim * BN);
     const long long n_lat = rnd((long long)c.latent_channels * BN), n_wav = rnd((long long)h->hop * BN);
     const long long nbuf = 1 + 2 * c.n_resblocks;
-    // tensor-core A operands: per block, heads and tails of B x C x (L + padding rows) bf16
-    int cmax_tc = 0;
-    for (int i = 0; i < c.n_stages; ++i)
-        if (h->stage_tc[i]) cmax_tc = std::max(cmax_tc, stage_channels(c, i));
-    h->a_cap = cmax_tc ? h->stage_cap + (long long)c.max_batch * cmax_tc * (kApadL + kApadR) : 0;
+    // tensor-core A operands: per block, heads and tails of B x C x (L + padding rows) bf16, for
+    // every layer that reads them (AMP convs, conv_pre, upsamplers)
+    {
+        long long need = 0, Lin = c.max_frames;
+        const long long pads = kApadL + kApadR;
+        if (h->pre_tc) need = std::max(need, (long long)c.latent_dim * (c.max_frames + pads));
+        int Cin = c.decoder_dim;
+        for (int i = 0; i < c.n_stages; ++i) {
+            if (h->ups_tc[i]) need = std::max(need, (long long)Cin * (Lin + pads));
+            Lin *= c.rates[i];
+            Cin /= 2;
+            if (h->stage_tc[i]) need = std::max(need, (long long)Cin * (Lin + pads));
+        }
+        h->a_cap = need * c.max_batch;
+    }
     const long long n_a = rnd((h->a_cap + 1) / 2);   // floats per head or tail array
     const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64 + 2 * c.n_resblocks * n_a;
     h->abytes = (size_t)total * sizeof(float);

@@ -77,5 +77,7 @@ struct DevAct {
 int launch_conv_simt(const ConvParams& p, int njobs, bool act, bool mean3, cudaStream_t s);
 int launch_convT_simt(const ConvTParams& p, bool mean3, cudaStream_t s);
 int launch_mean3(const Mean3Params& p, cudaStream_t s);
+// k = 1 conv with at most 64 input channels (the input projection); -1 if the shape does not fit.
+int launch_conv1x1(const ConvParams& p, cudaStream_t s);
 
 }  // namespace mh3a

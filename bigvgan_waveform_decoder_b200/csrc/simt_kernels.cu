@@ -454,6 +454,47 @@ int launch_convT_simt(const ConvTParams& p, bool mean3, cudaStream_t s) {
     return launch_convT_rate<8>(p, mean3, s);
 }
 
+// Pointwise (k = 1) conv with few input channels (dec_in_proj, 32 -> 2048): one thread per time
+// sample holds the Cin inputs in registers and sweeps 64 output channels whose weights sit in
+// shared memory (every lane reads the same weight: a broadcast).
+constexpr int kPwCin = 64;
+constexpr int kPwOut = 64;
+constexpr int kPwThreads = 128;
+
+__global__ void __launch_bounds__(kPwThreads) k_conv1x1(const ConvParams p) {
+    __shared__ float ws[kPwCin][kPwOut];
+    const ConvJob& J = p.job[0];
+    const int L = p.L, Cin = p.Cin, Cout = p.Cout;
+    const int tiles = (L + kPwThreads - 1) / kPwThreads;
+    const int b = blockIdx.x / tiles;
+    const int t = (blockIdx.x % tiles) * kPwThreads + threadIdx.x;
+    const int o0 = blockIdx.y * kPwOut;
+    for (int i = threadIdx.x; i < Cin * kPwOut; i += kPwThreads) {
+        const int c = i / kPwOut, o = i % kPwOut;
+        ws[c][o] = (o0 + o < Cout) ? __ldg(J.w + (size_t)c * Cout + o0 + o) : 0.f;   // [Cin, 1, Cout]
+    }
+    __syncthreads();
+    if (t >= L) return;
+    float z[kPwCin];
+#pragma unroll
+    for (int c = 0; c < kPwCin; ++c) z[c] = (c < Cin) ? __ldg(J.x0 + ((long long)b * Cin + c) * L + t) : 0.f;
+    for (int o = 0; o < kPwOut && o0 + o < Cout; ++o) {
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < kPwCin; ++c)
+            if (c < Cin) acc = fmaf(ws[c][o], z[c], acc);
+        J.out[((long long)b * Cout + o0 + o) * L + t] = acc + __ldg(J.bias + o0 + o);
+    }
+}
+
+int launch_conv1x1(const ConvParams& p, cudaStream_t s) {
+    const ConvJob& J = p.job[0];
+    if (J.K != 1 || J.pad != 0 || p.Cin < 1 || p.Cin > kPwCin || p.L < 1 || !J.bias) return -1;
+    dim3 grid(((p.L + kPwThreads - 1) / kPwThreads) * p.B, (p.Cout + kPwOut - 1) / kPwOut);
+    k_conv1x1<<<grid, kPwThreads, 0, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
+
 int launch_mean3(const Mean3Params& p, cudaStream_t s) {
     const int threads = 256;
     long long blocks = (p.n / 4 + threads - 1) / threads;

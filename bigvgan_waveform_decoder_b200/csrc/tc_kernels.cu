@@ -505,6 +505,10 @@ struct GemmJob {
     const float* res;
     float* out;
     int K, dil, pad;
+    int span;             // window rows a tile reads beyond its 128 MT output rows
+    // polyphase transposed conv (R > 1): window row offset and output phase of every tap
+    int8_t tap_row[16];
+    int8_t tap_phase[16];
 };
 
 struct GemmParams {
@@ -788,10 +792,15 @@ __device__ __forceinline__ int ps_tile_index(int i, int ntiles) {
     return k < ntiles ? k : -1;
 }
 
-template <int MT, int NT, int KGT, int EW>
+// R > 1: the polyphase transposed conv (upsampler).  Rows are input samples u; tap j reads the
+// window at row offset tap_row[j] and accumulates into the region of its output phase
+// tap_phase[j]; the epilogue writes phase phi of row u to output sample R u + phi.  A pass is
+// then one whole chunk, so that the first tap of every phase (j < R) starts its region.
+template <int MT, int NT, int KGT, int EW, int R>
 __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    static_assert(MT * NT <= PS_BUFCOLS, "one accumulator buffer holds MT x NT columns");
+    static_assert(R * MT * NT <= PS_BUFCOLS, "one accumulator buffer holds R x MT x NT columns");
+    static_assert(R == 1 || KGT >= 2, "the upsampler uses 16- or 32-channel chunks");
     static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
     static_assert(EW == 8 || EW == 16, "epilogue warps");
     static_assert((4 * MT * NT / EW) % 16 == 0 && 4 * MT * NT / EW <= NT, "epilogue column split");
@@ -845,86 +854,92 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
 
     if (warp == 0) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            // Descriptors are built once per ring slot and then advanced by adding 16-byte
-            // offsets to their low word (the start-address field), so that issuing an MMA costs
-            // a few integer adds: narrow tiles finish an MMA in 16 cycles.
-            constexpr uint32_t idesc = ptx::idesc_bf16(128, NT);
-            constexpr int KK = (KGT == 1) ? 1 : KGT / 2;   // K-steps per tap unit
-            const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
-            bool ok = *abort_flag == 0;
-            int sa = 0, sb = 0, buf = 0;
-            uint32_t pa = 0, pb = 0, pacc = 0;   // phase bits of the slots in use
-            for (int i = 0; ok; ++i) {
-                const int k = ps_tile_index(i, sc.ntiles);
-                if (k < 0) break;
-                const PsTile T = ps_tile<MT>(p, sc, k);
-                const GemmJob& J = p.job[T.z];
-                const int K = J.K, dil = J.dil;
-                const int KU = (KGT == 1) ? (K + 1) / 2 : K;
-                const uint32_t step = (uint32_t)((KGT == 1 ? 2 : 1) * dil);   // window rows per unit
-                const uint32_t a_lbo = (KGT == 1) ? (uint32_t)dil * 16 : (uint32_t)RS * 16;
-                for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
-                    if (!ptx::mbar_wait(&a_full[sa], pa, kWaitLimit)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t ah0 = ptx::desc_lo(a_smem + sa * pl.SA, a_lbo);
-                    int ucopy = 0, upass = 0;
-                    uint32_t bh0 = 0, ashift = 0;
-                    for (int unit = 0; unit < KU; ++unit, ashift += step) {
-                        if (ucopy == 0) {
-                            if (!ptx::mbar_wait(&b_full[sb], pb, kWaitLimit)) { ok = false; break; }
-                            ptx::tc_fence_after();
-                            bh0 = ptx::desc_lo(b_smem + sb * pl.SB, NT * 16);
-                        }
-                        if (upass == 0) {
-                            if (!ptx::mbar_wait(&acc_empty[buf], pacc ^ 1, kWaitLimit)) { ok = false; break; }
-                            ptx::tc_fence_after();
-                        }
-                        // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
-                        // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
-                        const uint32_t bh = bh0 + (uint32_t)ucopy * (TAPB >> 4);
-                        const uint32_t dbase = tmem + (uint32_t)(buf * PS_BUFCOLS);
+        // The whole warp walks the loop in lock step, so that every descriptor and address is
+        // warp-uniform; one elected lane issues each group of three MMAs and each commit.
+        // Descriptors are built once per ring slot and advanced by adding 16-byte offsets to
+        // their low word (the start-address field).
+        constexpr uint32_t idesc = ptx::idesc_bf16(128, NT);
+        constexpr int KK = (KGT == 1) ? 1 : KGT / 2;   // K-steps per tap unit
+        const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
+        bool ok = *abort_flag == 0;
+        int sa = 0, sb = 0, buf = 0;
+        uint32_t pa = 0, pb = 0, pacc = 0;   // phase bits of the slots in use
+        for (int i = 0; ok; ++i) {
+            const int k = ps_tile_index(i, sc.ntiles);
+            if (k < 0) break;
+            const PsTile T = ps_tile<MT>(p, sc, k);
+            const GemmJob& J = p.job[T.z];
+            const int K = J.K, dil = J.dil;
+            const int KU = (KGT == 1) ? (K + 1) / 2 : K;
+            const uint32_t step = (uint32_t)((KGT == 1 ? 2 : 1) * dil);   // window rows per unit
+            const uint32_t a_lbo = (KGT == 1) ? (uint32_t)dil * 16 : (uint32_t)RS * 16;
+            for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&a_full[sa], pa, kWaitLimit))) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t ah0 = ptx::desc_lo(a_smem + sa * pl.SA, a_lbo);
+                int ucopy = 0, upass = 0;
+                uint32_t bh0 = 0, ashift = 0;
+                for (int unit = 0; unit < KU; ++unit, ashift += step) {
+                    if (ucopy == 0) {
+                        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&b_full[sb], pb, kWaitLimit))) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        bh0 = ptx::desc_lo(b_smem + sb * pl.SB, NT * 16);
+                    }
+                    if (upass == 0) {
+                        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&acc_empty[buf], pacc ^ 1, kWaitLimit))) { ok = false; break; }
+                        ptx::tc_fence_after();
+                    }
+                    // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
+                    // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
+                    const uint32_t bh = bh0 + (uint32_t)ucopy * (TAPB >> 4);
+                    uint32_t dbase = tmem + (uint32_t)(buf * PS_BUFCOLS);
+                    uint32_t arow = ashift;
+                    bool first = upass == 0;
+                    if (R > 1) {
+                        arow = (uint32_t)J.tap_row[unit];
+                        dbase += (uint32_t)(J.tap_phase[unit] * NT);
+                        first = unit < R;
+                    }
 #pragma unroll
-                        for (int kk = 0; kk < KK; ++kk) {
-                            const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
-                            const uint32_t blk = bhk + (uint32_t)(BG * NT);
+                    for (int kk = 0; kk < KK; ++kk) {
+                        const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
+                        const uint32_t blk = bhk + (uint32_t)(BG * NT);
 #pragma unroll
-                            for (int mt = 0; mt < MT; ++mt) {
-                                const uint32_t a = ah0 + ashift + (uint32_t)(2 * kk * RS + mt * 128);
-                                const uint32_t d = dbase + (uint32_t)(mt * NT);
-                                ptx::mma_bf16(d, ptx::desc64(a), ptx::desc64(bhk), idesc, (upass == 0 && kk == 0) ? 0u : 1u);
-                                ptx::mma_bf16(d, ptx::desc64(a), ptx::desc64(blk), idesc, 1u);
-                                ptx::mma_bf16(d, ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bhk), idesc, 1u);
-                            }
-                        }
-                        ++ucopy;
-                        ++upass;
-                        if (ucopy == TPU || unit == KU - 1) {
-                            ptx::mma_commit(&b_empty[sb]);
-                            ucopy = 0;
-                            if (++sb == nsb) { sb = 0; pb ^= 1; }
-                        }
-                        if (upass == PU || unit == KU - 1) {
-                            ptx::mma_commit(&acc_full[buf]);
-                            upass = 0;
-                            buf ^= 1;
-                            if (buf == 0) pacc ^= 1;
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const uint32_t a = ah0 + arow + (uint32_t)(2 * kk * RS + mt * 128);
+                            ptx::mma3_bf16_elect(dbase + (uint32_t)(mt * R * NT), ptx::desc64(a),
+                                                 ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bhk),
+                                                 ptx::desc64(blk), idesc, (first && kk == 0) ? 0u : 1u);
                         }
                     }
-                    if (!ok) break;
-                    ptx::mma_commit(&a_empty[sa]);
-                    if (++sa == nsa) { sa = 0; pa ^= 1; }
-                    if (*abort_flag) ok = false;
+                    ++ucopy;
+                    ++upass;
+                    if (ucopy == TPU || unit == KU - 1) {
+                        ptx::mma_commit_elect(&b_empty[sb]);
+                        ucopy = 0;
+                        if (++sb == nsb) { sb = 0; pb ^= 1; }
+                    }
+                    if (upass == PU || unit == KU - 1) {
+                        ptx::mma_commit_elect(&acc_full[buf]);
+                        upass = 0;
+                        buf ^= 1;
+                        if (buf == 0) pacc ^= 1;
+                    }
                 }
+                if (!ok) break;
+                ptx::mma_commit_elect(&a_empty[sa]);
+                if (++sa == nsa) { sa = 0; pa ^= 1; }
+                if (*abort_flag) ok = false;
+                ok = __all_sync(0xffffffffu, ok);
             }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicExch(p.err, 5);
-            }
-            // every MMA issued has completed before the CTA releases its tensor memory
-            ptx::mma_commit(done_bar);
-            ptx::mbar_wait(done_bar, 0, kWaitLimit);
         }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(p.err, 5);
+        }
+        // every MMA issued has completed before the CTA releases its tensor memory
+        ptx::mma_commit_elect(done_bar);
+        ptx::mbar_wait(done_bar, 0, kWaitLimit);
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- A and B loader
@@ -937,10 +952,10 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                 if (k < 0) break;
                 const PsTile T = ps_tile<MT>(p, sc, k);
                 const GemmJob& J = p.job[T.z];
-                const int K = J.K, dil = J.dil;
+                const int K = J.K;
                 const int KU = (KGT == 1) ? (K + 1) / 2 : K;
                 const int NUC = (KU + TPU - 1) / TPU;
-                const int ROWS = 128 * MT + (K - 1) * dil + (KGT == 1 ? dil : 0);
+                const int ROWS = 128 * MT + J.span;
                 const uint32_t a_bytes = (uint32_t)(2 * KGT * ROWS * 16);
                 const long long row0 = p.pad_l + T.t0 - J.pad;   // first window row in the A arrays
                 const uint16_t* wsrc = J.w + (size_t)T.ot * nchunks * KU * unit_elems;
@@ -986,10 +1001,12 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         // ---------------------------------------------------------------- epilogue (warps 2 .. EW+1)
         const int e = warp - 2;
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
-        const int col0 = (e >> 2) * CW;        // first accumulator column of this warp
+        const int col0 = (e >> 2) * CW;        // first channel column of this warp ([mt][NT] order)
         const int mt = col0 / NT, oc0 = col0 % NT;
-        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)col0;
-        constexpr bool kPrefetch = CW <= 16;   // residual loaded ahead while the MMAs run
+        // regions [mt][phase][NT]: this warp's columns of phase phi start at + phi * NT
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(mt * R * NT + oc0);
+        constexpr bool kPrefetch = (R == 1) && CW <= 16;   // residual loaded ahead of the MMAs
+        const long long Lout = (long long)L * R;
         bool ok = *abort_flag == 0;
         int ip = 0;
         for (int i = 0; ok; ++i) {
@@ -999,28 +1016,31 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             const GemmJob& J = p.job[T.z];
             const int KU = (KGT == 1) ? (J.K + 1) / 2 : J.K;
             const int npass = nchunks * ((KU + PU - 1) / PU);
-            const int t = T.t0 + mt * 128 + q4 * 32 + lane;
+            const int t = T.t0 + mt * 128 + q4 * 32 + lane;   // the row (input sample when R > 1)
             const int o_base = T.ot * NT + oc0;
-            const long long idx0 = ((long long)T.b * Cout + o_base) * L + t;
+            const long long idx0 = ((long long)T.b * Cout + o_base) * Lout + (long long)R * t;
             float res[kPrefetch ? CW : 1];
             if (kPrefetch) {
 #pragma unroll
                 for (int c = 0; c < CW; ++c)
-                    res[c] = (J.res && t < L && o_base + c < Cout) ? J.res[idx0 + (long long)c * L] : 0.f;
+                    res[c] = (J.res && t < L && o_base + c < Cout) ? J.res[idx0 + (long long)c * Lout] : 0.f;
             }
-            float acc[CW];
+            float acc[R * CW];
 #pragma unroll
-            for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+            for (int c = 0; c < R * CW; ++c) acc[c] = 0.f;
             for (int ps = 0; ps < npass; ++ps, ++ip) {
                 const int buf = ip & 1;
                 if (!ptx::mbar_wait(&acc_full[buf], (ip >> 1) & 1, kWaitLimit)) { ok = false; break; }
                 ptx::tc_fence_after();
 #pragma unroll
-                for (int cb = 0; cb < CW; cb += 16) {
-                    float v[16];
-                    ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + cb), v);
+                for (int ph = 0; ph < R; ++ph) {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) acc[cb + c] += v[c];
+                    for (int cb = 0; cb < CW; cb += 16) {
+                        float v[16];
+                        ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) acc[ph * CW + cb + c] += v[c];
+                    }
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -1031,8 +1051,8 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                 break;
             }
             if (t < L) {
-                // FC columns at a time: all loads of a group are in flight before its stores
-                constexpr int FC = (CW > 64) ? 8 : 16;
+                // FC channels at a time: all loads of a group are in flight before its stores
+                constexpr int FC = (R * CW > 64) ? 8 : 16;
 #pragma unroll
                 for (int cb = 0; cb < CW; cb += FC) {
                     float bs[FC], rs[FC];
@@ -1041,11 +1061,15 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                         const int o = o_base + cb + c;   // channels past Cout pad the tile
                         bs[c] = (o < Cout) ? __ldg(J.bias + o) : 0.f;
                         if (kPrefetch) rs[c] = res[cb + c];
-                        else rs[c] = (J.res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * L] : 0.f;
+                        else rs[c] = (R == 1 && J.res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * Lout] : 0.f;
                     }
 #pragma unroll
-                    for (int c = 0; c < FC; ++c)
-                        if (o_base + cb + c < Cout) J.out[idx0 + (long long)(cb + c) * L] = (acc[cb + c] + bs[c]) + rs[c];
+                    for (int c = 0; c < FC; ++c) {
+                        if (o_base + cb + c >= Cout) continue;
+#pragma unroll
+                        for (int ph = 0; ph < R; ++ph)
+                            J.out[idx0 + (long long)(cb + c) * Lout + ph] = (acc[ph * CW + cb + c] + bs[c]) + rs[c];
+                    }
                 }
             }
         }
@@ -1083,8 +1107,11 @@ int ntile_amp(int C) { return C >= 128 ? 128 : (C >= 64 ? 64 : C); }
 int ntile_pre(int) { return 64; }
 int ntile_convt(int Cout, int r) {
     if (r > 2) return Cout >= 32 ? 32 : Cout;
-    return Cout >= 64 ? 64 : Cout;
+    return Cout >= 64 ? 64 : (Cout > 16 ? Cout : 16);   // narrow outputs padded to 16 columns
 }
+
+// 8-channel groups per K chunk of an upsampler: 32-channel chunks, or one 16-channel chunk.
+int kgt_convt(int Cin) { return Cin % 32 == 0 ? 4 : (Cin == 16 ? 2 : 0); }
 
 template <int MODE, int MT, int NT, int NIN>
 TcPlan make_plan(const TcParams& p, int njobs) {
@@ -1202,33 +1229,38 @@ int sm_count() {
     return cache[dev];
 }
 
-template <int MT, int NT, int KGT, int EW>
+// Every job must carry K, pad (window rows before a tile's first output row) and span (window
+// rows past its last); R > 1 jobs also their tap tables.
+template <int MT, int NT, int KGT, int EW, int R>
 int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     GemmParams p = p0;
     const int kc = 8 * KGT;
     if (p.Cin % kc != 0 || njobs < 1) return -1;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
-    int span = 0, padmax = 0, dilmax = 0, kumax = 1;
+    int span = 0, kumax = 1;
     for (int j = 0; j < njobs; ++j) {
-        span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
-        padmax = std::max(padmax, p.job[j].pad);
-        dilmax = std::max(dilmax, p.job[j].dil);
-        kumax = std::max(kumax, KGT == 1 ? (p.job[j].K + 1) / 2 : p.job[j].K);
+        const GemmJob& J = p.job[j];
+        if (J.pad < 0 || J.span < 0 || J.K < 1 || (R > 1 && J.K > 16)) return -1;
+        span = std::max(span, J.span);
+        kumax = std::max(kumax, KGT == 1 ? (J.K + 1) / 2 : J.K);
+        // every window row the tiles touch must exist in the A arrays
+        if (p.pad_l < J.pad ||
+            p.Lpad < (long long)p.pad_l - J.pad + (long long)p.tiles_t * 128 * MT + J.span)
+            return -1;
+        if (R > 1)
+            for (int k = 0; k < J.K; ++k)
+                if (J.tap_phase[k] < 0 || J.tap_phase[k] >= R || J.tap_row[k] < 0 || J.tap_row[k] > J.span) return -1;
     }
-    const int extra = (KGT == 1) ? dilmax : 0;   // the phantom tap of the last tap pair
-    // every window row the tiles touch must exist in the A arrays
-    if (p.pad_l < padmax ||
-        p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax + extra)
-        return -1;
     constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * NT * 16;
     p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));   // weight copies of about 16 KB
     PsSched sc{};
     sc.n_ot = (p.Cout + NT - 1) / NT;
     sc.per_job = p.B * p.tiles_t * sc.n_ot;
     sc.ntiles = njobs * sc.per_job;
-    sc.pu = (KGT == 4) ? 4 : 8;                             // 8 MMA K-steps per pass
+    // passes of 8 MMA K-steps; the upsampler's pass is one whole chunk
+    sc.pu = (R > 1) ? 64 : (KGT == 4) ? 4 : 8;
     PsPlan pl{};
-    pl.RS = 128 * MT + span + extra;
+    pl.RS = 128 * MT + span;
     pl.SA = 2 * KGT * pl.RS * 16;
     pl.SB = p.tpu * TAPB;
     constexpr int kBudget = 227 * 1024 - (8 * (4 * PS_MAXS + 5) + 16) - 64;
@@ -1245,7 +1277,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     if (smem_req > 227 * 1024) return -1;
     const int nsm = sm_count();
     if (nsm <= 0) return -1;
-    auto kern = k_gemm_ps<MT, NT, KGT, EW>;
+    auto kern = k_gemm_ps<MT, NT, KGT, EW, R>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_req) != cudaSuccess) return -1;
     const int grid = std::min(sc.ntiles, nsm);
     kern<<<grid, ps_threads(EW), smem_req, s>>>(p, sc, pl);
@@ -1254,13 +1286,13 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
 
 int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
-        case 256: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
-        case 128: return launch_gemm_ps<2, 128, 4, 8>(p, njobs, s);
-        case 64: return launch_gemm_ps<2, 64, 4, 16>(p, njobs, s);
-        case 32: return launch_gemm_ps<2, 32, 4, 16>(p, njobs, s);
-        case 16: return launch_gemm_ps<4, 16, 2, 16>(p, njobs, s);
-        case 8: return launch_gemm_ps<4, 16, 1, 16>(p, njobs, s);
+        case 512: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
+        case 256: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
+        case 128: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
+        case 64: return launch_gemm_ps<2, 64, 4, 16, 1>(p, njobs, s);
+        case 32: return launch_gemm_ps<2, 32, 4, 16, 1>(p, njobs, s);
+        case 16: return launch_gemm_ps<4, 16, 2, 16, 1>(p, njobs, s);
+        case 8: return launch_gemm_ps<4, 16, 1, 16, 1>(p, njobs, s);
         default: return -1;
     }
 }
@@ -1347,11 +1379,14 @@ bool tc_stage_supported(int C, const mh3a_config& c) {
 bool tc_pre_supported(int Cout, int Cin, int k) { return Cout % 64 == 0 && Cin % KC == 0 && Cin >= 7 * KC && k <= 15; }
 
 bool tc_convt_supported(int Cin, int Cout, int r, int K) {
-    if (Cin % KC != 0) return false;
+    const int kgt = kgt_convt(Cin);
+    if (kgt == 0) return false;
     if (r != 5 && r != 2) return false;
-    if (K > 16) return false;
+    if (K > 16 || K < r) return false;
     const int NT = ntile_convt(Cout, r);
-    if (NT < 16 || NT % 16 != 0 || Cout % NT != 0) return false;
+    if (NT < 16 || NT % 16 != 0 || (Cout % NT != 0 && Cout > NT)) return false;
+    if (r == 5 && (NT != 32 || kgt != 4)) return false;
+    if (kgt == 2 && NT != 16) return false;
     return true;
 }
 
@@ -1368,7 +1403,7 @@ void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWei
 
 void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
     pack_blocks([&](int o, int c, int tap) { return w_iok[((size_t)c * Cout + o) * K + tap]; }, Cout, Cin, K,
-                ntile_convt(Cout, r), KG, out);
+                ntile_convt(Cout, r), kgt_convt(Cin), out);
 }
 
 void tc_finalize(TcStageWeights* w) {
@@ -1430,6 +1465,10 @@ int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w,
         G.K = cp.job[j].K;
         G.dil = cp.job[j].dil;
         G.pad = cp.job[j].pad;
+        int NT, KGT;
+        amp_layout(cp.Cin, &NT, &KGT);
+        // KGT == 1 pairs taps: the phantom tap after the last one reads `dil` more rows
+        G.span = (G.K - 1) * G.dil + (KGT == 1 ? G.dil : 0);
     }
     return dispatch_gemm(p, njobs, s);
 }
@@ -1446,6 +1485,77 @@ int launch_conv_pre_tc(const ConvParams& cp, const TcStageWeights& w, cudaStream
     p.job[0] = make_job(cp.job[0], w.pre);
     // 7 head accumulators rotate over the 64 chunks of 2048 input channels
     return launch_tc<MODE_PLAIN, 1, 64, 8, 1>(p, 1, s);
+}
+
+int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
+                         int pad_l, long long Lpad, cudaStream_t s, int* err) {
+    if (!w.pre.dev || cp.Cout % ntile_pre(cp.Cout) != 0) return -1;
+    GemmParams p{};
+    p.Cin = cp.Cin;
+    p.Cout = cp.Cout;
+    p.L = cp.L;
+    p.B = cp.B;
+    p.pad_l = pad_l;
+    p.Lpad = Lpad;
+    p.err = err;
+    GemmJob& G = p.job[0];
+    G.a_hi = static_cast<const uint8_t*>(a_hi);
+    G.a_lo = static_cast<const uint8_t*>(a_lo);
+    G.w = reinterpret_cast<const uint16_t*>(w.pre.dev);
+    G.bias = cp.job[0].bias;
+    G.res = nullptr;
+    G.out = cp.job[0].out;
+    G.K = cp.job[0].K;
+    G.dil = cp.job[0].dil;
+    G.pad = cp.job[0].pad;
+    G.span = (G.K - 1) * G.dil;
+    return launch_gemm_ps<1, 64, 4, 16, 1>(p, 1, s);
+}
+
+int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,
+                      int pad_l, long long Lpad, cudaStream_t s, int* err) {
+    if (!w.ups.dev || q.K > 16 || q.K < q.r) return -1;
+    GemmParams p{};
+    p.Cin = q.Cin;
+    p.Cout = q.Cout;
+    p.L = q.Lin;
+    p.B = q.B;
+    p.pad_l = pad_l;
+    p.Lpad = Lpad;
+    p.err = err;
+    GemmJob& G = p.job[0];
+    // tap j serves output phase phi = (j - pad) mod r and reads input row u + (phi + pad - j) / r
+    int sh[16], smin = 1 << 20, smax = -(1 << 20);
+    for (int j = 0; j < q.K; ++j) {
+        const int phase = ((j - q.pad) % q.r + q.r) % q.r;
+        sh[j] = (phase + q.pad - j) / q.r;   // exact: phase + pad - j is a multiple of r
+        G.tap_phase[j] = (int8_t)phase;
+        smin = std::min(smin, sh[j]);
+        smax = std::max(smax, sh[j]);
+    }
+    for (int j = 0; j < q.K; ++j) G.tap_row[j] = (int8_t)(sh[j] - smin);
+    G.a_hi = static_cast<const uint8_t*>(a_hi);
+    G.a_lo = static_cast<const uint8_t*>(a_lo);
+    G.w = reinterpret_cast<const uint16_t*>(w.ups.dev);
+    G.bias = q.bias;
+    G.res = nullptr;
+    G.out = q.out;
+    G.K = q.K;
+    G.dil = 1;
+    G.pad = -smin;
+    G.span = smax - smin;
+    const int NT = ntile_convt(q.Cout, q.r);
+    if (kgt_convt(q.Cin) == 2) return (q.r == 2 && NT == 16) ? launch_gemm_ps<2, 16, 2, 8, 2>(p, 1, s) : -1;
+    if (q.r == 5 && NT == 32) return launch_gemm_ps<1, 32, 4, 8, 5>(p, 1, s);
+    if (q.r == 2) {
+        switch (NT) {
+            case 64: return launch_gemm_ps<2, 64, 4, 8, 2>(p, 1, s);
+            case 32: return launch_gemm_ps<2, 32, 4, 8, 2>(p, 1, s);
+            case 16: return launch_gemm_ps<2, 16, 4, 8, 2>(p, 1, s);
+            default: return -1;
+        }
+    }
+    return -1;
 }
 
 int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err) {

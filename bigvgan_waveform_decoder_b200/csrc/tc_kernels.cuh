@@ -60,4 +60,11 @@ int launch_amp_gemm_tc(const ConvParams& p, int njobs, const TcStageWeights& w, 
 int launch_conv_pre_tc(const ConvParams& p, const TcStageWeights& w, cudaStream_t s, int* err);
 int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err);
 
+// conv_pre and the upsamplers on the persistent GEMM, reading their input as pre-split rows
+// (launch_split_rows) with pad_l zero rows before the sequence and Lpad rows per channel group.
+int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
+                         int pad_l, long long Lpad, cudaStream_t s, int* err);
+int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,
+                      int pad_l, long long Lpad, cudaStream_t s, int* err);
+
 }  // namespace mh3a

@@ -129,6 +129,33 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// One 3xBF16 K-step, issued by one elected lane of a converged warp: D (+)= Ah Bh, then
+// D += Ah Bl and D += Al Bh.  `accumulate` = 0 starts the accumulator with the first product.
+// Called by all 32 lanes with identical operands (computed in warp-uniform code).
+__device__ __forceinline__ void mma3_bf16_elect(uint32_t d_tmem, uint64_t ah, uint64_t al, uint64_t bh,
+                                                uint64_t bl, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, q;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "setp.eq.b32 q, %6, %6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %4, %5, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %3, %5, q;\n\t}" ::"r"(d_tmem),
+        "l"(ah), "l"(al), "l"(bh), "l"(bl), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// tcgen05.commit by one elected lane of a converged warp.
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
