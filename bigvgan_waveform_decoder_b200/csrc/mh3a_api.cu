@@ -130,7 +130,8 @@ struct mh3a_handle {
     long long a_cap = 0;                   // bf16 elements per A array
     float* lat_io = nullptr;   // host-API staging
     float* wav_io = nullptr;
-    int* dev_err = nullptr;    // set by a tensor-core kernel whose bounded wait timed out
+    int* dev_err = nullptr;    // 64 ints: [0] set by a tensor-core kernel whose bounded wait timed
+                               // out; [16..17] the persistent GEMM's tile scheduler
     // profiling
     bool profiling = false;
     cudaEvent_t ev[kMaxSegments + 1] = {};
@@ -338,7 +339,7 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                 mh3a_status st = counted(h, launch_act_split(ap, nrb, s));
                 if (st) return st;
                 const long long Lpad = (long long)L + kApadL + kApadR;
-                n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err);
+                n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err, h->dev_err + 16);
             } else {
                 n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             }
@@ -411,7 +412,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             // split the input into head/tail rows once, then the persistent tensor-core GEMM
             if ((st = split_to_a(h, h->buf_in, nullptr, nullptr, c.latent_dim, N, B, s))) return st;
             n = launch_conv_pre_gemm(p, h->tc[0], h->A_hi[0], h->A_lo[0], kApadL, (long long)N + kApadL + kApadR,
-                                     s, h->dev_err);
+                                     s, h->dev_err, h->dev_err + 16);
         } else {
             n = launch_conv_simt(p, 1, false, false, s);
         }
@@ -443,7 +444,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         if (h->ups_tc[i]) {
             if ((st = split_to_a(h, q.x0, q.x1, q.x2, C, L, B, s))) return st;
             nl = launch_convT_gemm(q, h->tc[i], h->A_hi[0], h->A_lo[0], kApadL, (long long)L + kApadL + kApadR, s,
-                                   h->dev_err);
+                                   h->dev_err, h->dev_err + 16);
         } else {
             nl = launch_convT_simt(q, mean3, s);
         }
@@ -851,7 +852,8 @@ mh3a_status mh3a_check_device_error(mh3a_handle* h) {
     int flag = 0;
     CK_CUDA(cudaMemcpy(&flag, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost), "read device error flag");
     if (flag == 0) return MH3A_OK;
-    CK_CUDA(cudaMemset(h->dev_err, 0, sizeof(int)), "clear device error flag");
+    // the flag and the tile scheduler's counters (stale after an aborted launch)
+    CK_CUDA(cudaMemset(h->dev_err, 0, 64 * sizeof(int)), "clear device error flag");
     g_last_error = "a tensor-core kernel gave up waiting on its pipeline (code " + std::to_string(flag) +
                    "); its outputs are invalid";
     return MH3A_ERR_CUDA;

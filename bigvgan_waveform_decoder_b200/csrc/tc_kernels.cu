@@ -489,13 +489,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
 }
 
 // ----------------------------------------------------------------------------------------------
-// GEMM-only variant for the AMP convolutions: the activation has already been written to
-// memory as the A operand (rows of 8 bf16 channels, heads and tails in separate arrays, with
-// the conv's zero padding materialised), so both operands arrive by 1-D bulk copies and the
-// kernel needs only the MMA warp, the loader warp and 4 epilogue warps.
+// GEMM operands for the persistent kernel below: the activation (or plain split) has already
+// been written to memory as the A operand (rows of 8 bf16 channels, heads and tails in separate
+// arrays, with the conv's zero padding materialised), so both operands arrive by 1-D bulk
+// copies.
 // ----------------------------------------------------------------------------------------------
-
-constexpr int GEMM_THREADS = 192;   // warp 0 MMA, warp 1 loader, warps 2..5 epilogue
 
 struct GemmJob {
     const uint8_t* a_hi;   // [B, Cin/8, Lpad] rows of 16 bytes
@@ -518,223 +516,8 @@ struct GemmParams {
     long long Lpad;       // rows per (item, channel group) in the A arrays
     int tpu;              // tap units per weight bulk copy (set by the launcher)
     int* err;
+    int* sched;           // [next tile, CTAs done]: zero before a launch, left zero after it
 };
-
-// KGT = 8-channel groups per K chunk (4: 32 input channels; 2: 16).  KGT = 1 serves 8-channel
-// layers: one MMA K-step of 16 then covers the same 8 channels at two consecutive taps -- the
-// second core matrix along K is the window shifted by `dil` rows, i.e. the A descriptor's
-// leading-byte offset is dil * 16 -- and the weight block of a unit holds that tap pair (a
-// zero block stands in for the tap past the last one).
-template <int MT, int NT, int NACC, int KGT>
-__global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p, const TcPlan pl) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    constexpr int NHH = NACC - 1;
-    constexpr int USED = MT * NT * NACC;
-    static_assert(NACC >= 2 && USED <= 512, "tensor memory holds 512 columns");
-    static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
-    constexpr int NCOLS = (USED <= 32) ? 32 : (USED <= 64) ? 64 : (USED <= 128) ? 128 : (USED <= 256) ? 256 : 512;
-    constexpr int BG = (KGT == 1) ? 2 : KGT;   // core-matrix columns (K) per weight block part
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const GemmJob& J = p.job[blockIdx.z];
-    const int K = J.K, dil = J.dil, pad = J.pad;
-    const int Cin = p.Cin, Cout = p.Cout, L = p.L;
-    const int b = blockIdx.x / p.tiles_t;
-    const int t0 = (blockIdx.x % p.tiles_t) * (128 * MT);
-    const int o_tile = blockIdx.y;
-    const int o0 = o_tile * NT;
-    const int nchunks = Cin / (8 * KGT);
-    const int KU = (KGT == 1) ? (K + 1) / 2 : K;            // tap units (taps or tap pairs) per chunk
-    const int TPU = p.tpu;                                   // tap units per weight copy
-    const int NUC = (KU + TPU - 1) / TPU;                    // weight copies per chunk
-    constexpr int TAPB = 2 * BG * NT * 16;                   // bytes of one tap unit (head + tail)
-    const int ROWS = 128 * MT + (K - 1) * dil + (KGT == 1 ? dil : 0);
-    const int RS = pl.RS;
-
-    uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
-    uint8_t* Bs = smem + pl.offB;              // [NSB][2][KG][NT][16 B]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
-    uint64_t* a_full = bars;
-    uint64_t* a_empty = bars + NSA;
-    uint64_t* b_full = bars + 2 * NSA;
-    uint64_t* b_empty = bars + 2 * NSA + NSB;
-    uint64_t* acc_full = bars + 2 * NSA + 2 * NSB;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSA + 2 * NSB + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* epi_go = abort_flag + 1;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NSA; ++s) {
-            ptx::mbar_init(&a_full[s], 1);
-            ptx::mbar_init(&a_empty[s], 1);
-        }
-        for (int s = 0; s < NSB; ++s) {
-            ptx::mbar_init(&b_full[s], 1);
-            ptx::mbar_init(&b_empty[s], 1);
-        }
-        ptx::mbar_init(acc_full, 1);
-        *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
-        *epi_go = 0;
-        ptx::fence_mbar_init();
-    }
-    if (warp == 0) {
-        ptx::tmem_alloc(tmem_slot, NCOLS);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = ptx::idesc_bf16(128, NT);
-            const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
-            const bool skip = *abort_flag != 0;
-            bool ok = !skip;
-            int u = 0;
-            for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
-                const int sa = chunk % NSA;
-                if (!ptx::mbar_wait(&a_full[sa], (chunk / NSA) & 1, kWaitLimit)) { ok = false; break; }
-                ptx::tc_fence_after();
-                const uint32_t a_hi = a_smem + sa * pl.SA;
-                const uint32_t a_lo = a_hi + KGT * RS * 16;
-                for (int uc = 0; uc < NUC; ++uc, ++u) {
-                    const int sb = u % NSB;
-                    if (!ptx::mbar_wait(&b_full[sb], (u / NSB) & 1, kWaitLimit)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const int ut_end = min(KU, (uc + 1) * TPU);
-                    for (int unit = uc * TPU; unit < ut_end; ++unit) {
-                    const uint32_t b_hi = b_smem + sb * pl.SB + (unit - uc * TPU) * TAPB;
-                    const uint32_t b_lo = b_hi + BG * NT * 16;
-                    // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
-                    // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
-                    const int row_shift = (KGT == 1 ? 2 * unit : unit) * dil;
-                    const uint32_t a_lbo = (KGT == 1) ? (uint32_t)dil * 16 : (uint32_t)RS * 16;
-#pragma unroll
-                    for (int kk = 0; kk < (KGT == 1 ? 1 : KGT / 2); ++kk) {
-                        const uint32_t boff = (uint32_t)(2 * kk) * NT * 16;
-                        const uint64_t bh = ptx::smem_desc(b_hi + boff, NT * 16, 128);
-                        const uint64_t bl = ptx::smem_desc(b_lo + boff, NT * 16, 128);
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + row_shift) * 16;
-                            const uint64_t ah = ptx::smem_desc(a_hi + aoff, a_lbo, 128);
-                            const uint64_t al = ptx::smem_desc(a_lo + aoff, a_lbo, 128);
-                            const int accbase = mt * NACC;
-                            const uint32_t dh = tmem + (uint32_t)((accbase + chunk % NHH) * NT);
-                            const uint32_t dx = tmem + (uint32_t)((accbase + NHH) * NT);
-                            const uint32_t acc_h = (chunk >= NHH || unit > 0 || kk > 0) ? 1u : 0u;
-                            const uint32_t acc_x = (chunk > 0 || unit > 0 || kk > 0) ? 1u : 0u;
-                            ptx::mma_bf16(dh, ah, bh, idesc, acc_h);
-                            ptx::mma_bf16(dx, ah, bl, idesc, acc_x);
-                            ptx::mma_bf16(dx, al, bh, idesc, 1u);
-                        }
-                    }
-                    }
-                    ptx::mma_commit(&b_empty[sb]);
-                }
-                if (ok) ptx::mma_commit(&a_empty[sa]);
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                if (!skip) atomicExch(p.err, 5);
-            }
-            ptx::mma_commit(acc_full);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- A and B loader
-        if (lane == 0) {
-            const size_t unit_elems = (size_t)2 * BG * NT * 8;
-            const uint16_t* wsrc = J.w + (size_t)o_tile * nchunks * KU * unit_elems;
-            const uint32_t a_bytes = (uint32_t)(2 * KGT * ROWS * 16);
-            const long long row0 = p.pad_l + t0 - pad;   // first window row in the A arrays
-            int a_issued = 0, b_issued = 0, u = 0;
-            bool ok = *abort_flag == 0;
-            for (int chunk = 0; chunk < nchunks && ok; ++chunk) {
-                const int sa = chunk % NSA;
-                if (!ptx::mbar_wait(&a_empty[sa], ((chunk / NSA) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                ptx::mbar_arrive_expect_tx(&a_full[sa], a_bytes);
-                for (int part = 0; part < 2; ++part) {
-                    const uint8_t* base = part == 0 ? J.a_hi : J.a_lo;
-                    for (int g = 0; g < KGT; ++g) {
-                        const long long grp = (long long)b * (Cin / 8) + chunk * KGT + g;
-                        ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KGT + g) * RS) * 16,
-                                      base + (grp * p.Lpad + row0) * 16, (uint32_t)(ROWS * 16), &a_full[sa]);
-                    }
-                }
-                a_issued = chunk + 1;
-                for (int uc = 0; uc < NUC; ++uc, ++u) {
-                    const int sb = u % NSB;
-                    if (!ptx::mbar_wait(&b_empty[sb], ((u / NSB) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                    // tap units [uc * TPU, min(KU, (uc + 1) * TPU)) are contiguous in the packing
-                    const int nunits = min(KU, (uc + 1) * TPU) - uc * TPU;
-                    const uint32_t bytes = (uint32_t)(nunits * TAPB);
-                    ptx::mbar_arrive_expect_tx(&b_full[sb], bytes);
-                    ptx::bulk_g2s(Bs + (size_t)sb * pl.SB, wsrc + ((size_t)chunk * KU + (size_t)uc * TPU) * unit_elems,
-                                  bytes, &b_full[sb]);
-                    b_issued = u + 1;
-                }
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicExch(p.err, 6);
-                // let the copies already in flight land before the CTA can exit
-                for (int c = (a_issued > NSA ? a_issued - NSA : 0); c < a_issued; ++c)
-                    ptx::mbar_wait(&a_full[c % NSA], (c / NSA) & 1, kWaitLimit);
-                for (int v = (b_issued > NSB ? b_issued - NSB : 0); v < b_issued; ++v)
-                    ptx::mbar_wait(&b_full[v % NSB], (v / NSB) & 1, kWaitLimit);
-            }
-        }
-        __syncwarp();
-    } else {
-        // ---------------------------------------------------------------- epilogue (warps 2..5)
-        if (threadIdx.x == 64) {
-            bool go = ptx::mbar_wait(acc_full, 0, kWaitLimit);
-            if (!go) atomicExch(p.err, 7);
-            go = go && *abort_flag == 0;
-            *epi_go = go ? 1 : 0;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        const bool go = *epi_go != 0;   // identical in all four epilogue warps
-        ptx::tc_fence_after();
-        const int q4 = warp & 3;        // TMEM lane quarter this warp may access
-        const long long obase = (long long)b * Cout * L;
-        if (go) {
-            const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int t = t0 + mt * 128 + q4 * 32 + lane;
-                for (int cb = 0; cb < NT; cb += 16) {
-                    float v[16], w[16];
-                    ptx::tmem_ld16(lane_addr + (uint32_t)(mt * NACC * NT + cb), v);
-#pragma unroll
-                    for (int a = 1; a < NACC; ++a) {
-                        ptx::tmem_ld16(lane_addr + (uint32_t)((mt * NACC + a) * NT + cb), w);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] += w[i];
-                    }
-                    if (t < L) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int o = o0 + cb + i;
-                            if (o >= Cout) break;   // output channels padded up to the tile width
-                            const long long idx = obase + (long long)o * L + t;
-                            float y = v[i] + __ldg(J.bias + o);
-                            if (J.res) y += J.res[idx];
-                            J.out[idx] = y;
-                        }
-                    }
-                }
-            }
-        }
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    if (warp == 0) ptx::tmem_dealloc(tmem, NCOLS);
-}
 
 // ----------------------------------------------------------------------------------------------
 // persistent AMP GEMM: one CTA per SM walks a list of output tiles (job, item, 128 MT time rows,
@@ -748,6 +531,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) k_gemm_tc(const GemmParams p,
 // EW epilogue warps (EW / 4 per TMEM lane quarter) after warp 0 (MMA) and warp 1 (loader).
 constexpr int ps_threads(int EW) { return 64 + 32 * EW; }
 constexpr int PS_MAXS = 8;                              // ring stages (max)
+constexpr int PS_TQ = 16;                               // tile-index queue entries
 constexpr int PS_BUFCOLS = 256;                         // TMEM columns per accumulator buffer
 
 struct PsPlan {
@@ -782,16 +566,12 @@ __device__ __forceinline__ PsTile ps_tile(const GemmParams& p, const PsSched& sc
     return T;
 }
 
-// The i-th tile of this CTA: rounds of gridDim.x tiles, walked forwards and backwards in turn
-// so that a CTA that drew a heavy tile in one round draws a light one in the next.
-__device__ __forceinline__ int ps_tile_index(int i, int ntiles) {
-    const int G = gridDim.x;
-    const int base = i * G;
-    if (base >= ntiles) return -1;
-    const int k = base + ((i & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
-    return k < ntiles ? k : -1;
-}
 
+// KGT = 8-channel groups per K chunk (4: 32 input channels; 2: 16).  KGT = 1 serves 8-channel
+// layers: one MMA K-step of 16 then covers the same 8 channels at two consecutive taps -- the
+// second core matrix along K is the window shifted by `dil` rows, i.e. the A descriptor's
+// leading-byte offset is dil * 16 -- and the weight block of a unit holds that tap pair (a
+// zero block stands in for the tap past the last one).
 // R > 1: the polyphase transposed conv (upsampler).  Rows are input samples u; tap j reads the
 // window at row offset tap_row[j] and accumulates into the region of its output phase
 // tap_phase[j]; the epilogue writes phase phi of row u to output sample R u + phi.  A pass is
@@ -823,8 +603,10 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
     uint64_t* acc_full = bars + 4 * PS_MAXS;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* done_bar = acc_full + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    uint64_t* tile_full = done_bar + 1;                  // [PS_TQ] a tile index was queued
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_full + PS_TQ);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* tile_q = abort_flag + 1;               // [PS_TQ] tile indices, -1 = no more
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nsa; ++s) {
@@ -840,6 +622,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             ptx::mbar_init(&acc_empty[s], EW);
         }
         ptx::mbar_init(done_bar, 1);
+        for (int q = 0; q < PS_TQ; ++q) ptx::mbar_init(&tile_full[q], 1);
         *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
         ptx::fence_mbar_init();
     }
@@ -865,7 +648,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         int sa = 0, sb = 0, buf = 0;
         uint32_t pa = 0, pb = 0, pacc = 0;   // phase bits of the slots in use
         for (int i = 0; ok; ++i) {
-            const int k = ps_tile_index(i, sc.ntiles);
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tile_full[i % PS_TQ], (i / PS_TQ) & 1, kWaitLimit))) {
+                ok = false;
+                break;
+            }
+            const int k = tile_q[i % PS_TQ];
             if (k < 0) break;
             const PsTile T = ps_tile<MT>(p, sc, k);
             const GemmJob& J = p.job[T.z];
@@ -947,9 +734,17 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             const size_t unit_elems = (size_t)2 * BG * NT * 8;
             bool ok = *abort_flag == 0;
             int ia = 0, ib = 0;
+            bool drained = false;   // the scheduler handed this CTA its end marker
             for (int i = 0; ok; ++i) {
-                const int k = ps_tile_index(i, sc.ntiles);
-                if (k < 0) break;
+                // dynamic schedule: tiles go out heaviest job first, each to the CTA that asks next
+                int k = atomicAdd(p.sched, 1);
+                if (k >= sc.ntiles) k = -1;
+                tile_q[i % PS_TQ] = k;
+                ptx::mbar_arrive(&tile_full[i % PS_TQ]);
+                if (k < 0) {
+                    drained = true;
+                    break;
+                }
                 const PsTile T = ps_tile<MT>(p, sc, k);
                 const GemmJob& J = p.job[T.z];
                 const int K = J.K;
@@ -990,6 +785,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                 *abort_flag = 1;
                 atomicExch(p.err, 6);
             }
+            // the last CTA to drain the schedule resets it for the next launch
+            if (drained && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+                atomicExch(p.sched, 0);
+                atomicExch(p.sched + 1, 0);
+            }
             // let the copies still in flight land before the CTA can exit
             for (int c = (ia > nsa ? ia - nsa : 0); c < ia; ++c)
                 ptx::mbar_wait(&a_full[c % nsa], (c / nsa) & 1, kWaitLimit);
@@ -1010,7 +810,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         bool ok = *abort_flag == 0;
         int ip = 0;
         for (int i = 0; ok; ++i) {
-            const int k = ps_tile_index(i, sc.ntiles);
+            if (!ptx::mbar_wait(&tile_full[i % PS_TQ], (i / PS_TQ) & 1, kWaitLimit)) {
+                ok = false;
+                break;
+            }
+            const int k = tile_q[i % PS_TQ];
             if (k < 0) break;
             const PsTile T = ps_tile<MT>(p, sc, k);
             const GemmJob& J = p.job[T.z];
@@ -1103,7 +907,7 @@ float bf16_value(uint16_t h) {
 }
 
 // Output-channel tile of each layer kind (the weight blocks are laid out for it).
-int ntile_amp(int C) { return C >= 128 ? 128 : (C >= 64 ? 64 : C); }
+int ntile_amp(int C) { return C >= 256 ? 256 : (C >= 128 ? 128 : (C >= 64 ? 64 : C)); }
 int ntile_pre(int) { return 64; }
 int ntile_convt(int Cout, int r) {
     if (r > 2) return Cout >= 32 ? 32 : Cout;
@@ -1162,14 +966,14 @@ int launch_tc(const TcParams& p0, int njobs, cudaStream_t s) {
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
 
-// AMP tile shape per width: MT x 128 time rows, NT output channels, NACC accumulators per
-// M tile (MT * NT * NACC <= 512 tensor-memory columns).  The two widest stages use 128-column
-// tiles so that three head accumulators share their long K loops (accuracy: the accumulation
-// bias of these stages dominated the decode error with a single head accumulator).
+// Fused AMP kernel (allocation-free stage entry point): MT x 128 time rows, NT output channels,
+// NACC accumulators per M tile (MT * NT * NACC <= 512 tensor-memory columns).  NT follows the
+// weight packing shared with the persistent GEMM, so the two widest stages get 256-column tiles
+// and a single head accumulator (stage-0 relative error about 4e-5, against 1e-5 with three).
 int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
-        case 256: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
+        case 512: return launch_tc<MODE_AMP, 1, 256, 2, 1>(p, njobs, s);
+        case 256: return launch_tc<MODE_AMP, 1, 256, 2, 1>(p, njobs, s);
         case 128: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
         case 64: return launch_tc<MODE_AMP, 2, 64, 3, 1>(p, njobs, s);
         case 32: return launch_tc<MODE_AMP, 2, 32, 2, 1>(p, njobs, s);
@@ -1177,46 +981,6 @@ int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
     }
 }
 
-template <int MT, int NT, int NACC, int KGT>
-int launch_gemm(const GemmParams& p0, int njobs, cudaStream_t s) {
-    GemmParams p = p0;
-    const int kc = 8 * KGT;
-    if (NACC - 1 > p.Cin / kc || p.Cin % kc != 0) return -1;
-    p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
-    int span = 0, padmax = 0, dilmax = 0;
-    for (int j = 0; j < njobs; ++j) {
-        span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
-        padmax = std::max(padmax, p.job[j].pad);
-        dilmax = std::max(dilmax, p.job[j].dil);
-    }
-    const int extra = (KGT == 1) ? dilmax : 0;   // the phantom tap of the last tap pair
-    // every window row the tiles touch must exist in the A arrays
-    if (p.pad_l < padmax ||
-        p.Lpad < (long long)p.pad_l + (long long)p.tiles_t * 128 * MT + padmax + extra)
-        return -1;
-    // weight copies of about 16 KB: one L2 round trip then feeds several taps' MMAs
-    constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * NT * 16;
-    int kumax = 1;
-    for (int j = 0; j < njobs; ++j) kumax = std::max(kumax, KGT == 1 ? (p.job[j].K + 1) / 2 : p.job[j].K);
-    p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));
-    TcPlan pl{};
-    pl.RS = 128 * MT + span + extra;
-    pl.SA = 2 * KGT * pl.RS * 16;
-    // ... but not at the cost of the second CTA per SM (2 x 113 KB of shared memory)
-    while (p.tpu > 1 && NSA * pl.SA + NSB * p.tpu * TAPB + 1024 > 113 * 1024) --p.tpu;
-    pl.SB = p.tpu * TAPB;
-    pl.offB = NSA * pl.SA;
-    pl.offBar = (pl.offB + NSB * pl.SB + 15) / 16 * 16;
-    pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
-    if (pl.smem > 227 * 1024) return -1;
-    auto kern = k_gemm_tc<MT, NT, NACC, KGT>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess) return -1;
-    dim3 grid(p.tiles_t * p.B, (p.Cout + NT - 1) / NT, njobs);
-    kern<<<grid, GEMM_THREADS, pl.smem, s>>>(p, pl);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
-}
-
-// GEMM tile shape per width; NT and the channels per chunk must match amp_layout().
 int sm_count() {
     static int cache[64] = {};
     int dev = 0;
@@ -1235,7 +999,7 @@ template <int MT, int NT, int KGT, int EW, int R>
 int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     GemmParams p = p0;
     const int kc = 8 * KGT;
-    if (p.Cin % kc != 0 || njobs < 1) return -1;
+    if (p.Cin % kc != 0 || njobs < 1 || !p.sched || !p.err) return -1;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
     int span = 0, kumax = 1;
     for (int j = 0; j < njobs; ++j) {
@@ -1263,14 +1027,15 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     pl.RS = 128 * MT + span;
     pl.SA = 2 * KGT * pl.RS * 16;
     pl.SB = p.tpu * TAPB;
-    constexpr int kBudget = 227 * 1024 - (8 * (4 * PS_MAXS + 5) + 16) - 64;
+    constexpr int kBarBytes = 8 * (4 * PS_MAXS + 5 + PS_TQ) + 8 + 4 * PS_TQ;
+    constexpr int kBudget = 227 * 1024 - kBarBytes - 64;
     pl.nsa = (4 * pl.SA <= kBudget / 2) ? 4 : 3;
     if (pl.nsa * pl.SA + 2 * pl.SB > kBudget) pl.nsa = 2;
     pl.nsb = std::min(PS_MAXS, (kBudget - pl.nsa * pl.SA) / pl.SB);
     if (pl.nsb < 2) return -1;
     pl.offB = pl.nsa * pl.SA;
     pl.offBar = (pl.offB + pl.nsb * pl.SB + 15) / 16 * 16;
-    pl.smem = pl.offBar + 8 * (4 * PS_MAXS + 5) + 16;
+    pl.smem = pl.offBar + kBarBytes;
     // at least half the SM's shared memory, so that a second CTA never waits on the first's
     // tensor memory
     const int smem_req = std::max(pl.smem, 116 * 1024);
@@ -1286,8 +1051,8 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
 
 int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
-        case 256: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
+        case 512: return launch_gemm_ps<1, 256, 4, 8, 1>(p, njobs, s);
+        case 256: return launch_gemm_ps<1, 256, 4, 8, 1>(p, njobs, s);
         case 128: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
         case 64: return launch_gemm_ps<2, 64, 4, 16, 1>(p, njobs, s);
         case 32: return launch_gemm_ps<2, 32, 4, 16, 1>(p, njobs, s);
@@ -1438,8 +1203,9 @@ int launch_conv_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int
 
 int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int m, int half,
                        const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
-                       cudaStream_t s, int* err) {
+                       cudaStream_t s, int* err, int* sched) {
     GemmParams p{};
+    p.sched = sched;
     p.Cin = cp.Cin;
     p.Cout = cp.Cout;
     p.L = cp.L;
@@ -1473,24 +1239,12 @@ int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w,
     return dispatch_gemm(p, njobs, s);
 }
 
-int launch_conv_pre_tc(const ConvParams& cp, const TcStageWeights& w, cudaStream_t s, int* err) {
-    if (!w.pre.dev || cp.job[0].K > 15) return -1;
-    TcParams p{};
-    p.Cin = cp.Cin;
-    p.Cout = cp.Cout;
-    p.L = cp.L;
-    p.B = cp.B;
-    p.r = 1;
-    p.err = err;
-    p.job[0] = make_job(cp.job[0], w.pre);
-    // 7 head accumulators rotate over the 64 chunks of 2048 input channels
-    return launch_tc<MODE_PLAIN, 1, 64, 8, 1>(p, 1, s);
-}
 
 int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                         int pad_l, long long Lpad, cudaStream_t s, int* err) {
+                         int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched) {
     if (!w.pre.dev || cp.Cout % ntile_pre(cp.Cout) != 0) return -1;
     GemmParams p{};
+    p.sched = sched;
     p.Cin = cp.Cin;
     p.Cout = cp.Cout;
     p.L = cp.L;
@@ -1513,9 +1267,10 @@ int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const vo
 }
 
 int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                      int pad_l, long long Lpad, cudaStream_t s, int* err) {
+                      int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched) {
     if (!w.ups.dev || q.K > 16 || q.K < q.r) return -1;
     GemmParams p{};
+    p.sched = sched;
     p.Cin = q.Cin;
     p.Cout = q.Cout;
     p.L = q.Lin;
@@ -1558,55 +1313,5 @@ int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void*
     return -1;
 }
 
-int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err) {
-    if (!w.ups.dev) return -1;
-    TcParams p{};
-    p.Cin = q.Cin;
-    p.Cout = q.Cout;
-    p.L = q.Lin;
-    p.B = q.B;
-    p.r = q.r;
-    p.err = err;
-    // window rows before the tile: minus the smallest tap shift floor((phi + pad - j) / r)
-    int smin = 1000000;
-    for (int j = 0; j < q.K; ++j) {
-        const int phase = ((j - q.pad) % q.r + q.r) % q.r;
-        const int a = phase + q.pad - j;
-        smin = std::min(smin, a >= 0 ? a / q.r : -((-a + q.r - 1) / q.r));
-    }
-    p.lo = -smin;
-    TcJob& T = p.job[0];
-    T.x0 = q.x0;
-    T.x1 = q.x1;
-    T.x2 = q.x2;
-    T.w = reinterpret_cast<const uint16_t*>(w.ups.dev);
-    T.bias = q.bias;
-    T.out = q.out;
-    T.K = q.K;
-    T.dil = 1;
-    T.pad = q.pad;
-    // as many head accumulators per phase as tensor memory (and the chunk count) allow
-    const int NT = ntile_convt(q.Cout, q.r);
-    const int nchunks = q.Cin / KC;
-    if (q.r == 5) {
-        switch (NT) {
-            case 32: return nchunks >= 2 ? launch_tc<MODE_CONVT, 1, 32, 3, 5>(p, 1, s)
-                                         : launch_tc<MODE_CONVT, 1, 32, 2, 5>(p, 1, s);
-            case 16: return launch_tc<MODE_CONVT, 1, 16, 2, 5>(p, 1, s);
-            default: return -1;
-        }
-    }
-    if (q.r == 2) {
-        switch (NT) {
-            case 128: return launch_tc<MODE_CONVT, 1, 128, 2, 2>(p, 1, s);
-            case 64: return nchunks >= 3 ? launch_tc<MODE_CONVT, 1, 64, 4, 2>(p, 1, s)
-                                         : launch_tc<MODE_CONVT, 1, 64, 2, 2>(p, 1, s);
-            case 32: return launch_tc<MODE_CONVT, 1, 32, 2, 2>(p, 1, s);
-            case 16: return launch_tc<MODE_CONVT, 1, 16, 2, 2>(p, 1, s);
-            default: return -1;
-        }
-    }
-    return -1;
-}
 
 }  // namespace mh3a

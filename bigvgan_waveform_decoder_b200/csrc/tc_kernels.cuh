@@ -53,18 +53,17 @@ int launch_conv_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int 
                    cudaStream_t s, int* err);
 // The same layer as a pure GEMM whose A operand (the activation, heads and tails) has been
 // written by launch_act_split into a_hi[j] / a_lo[j] with pad_l zero rows before the sequence
-// and Lpad rows per (item, channel group).
+// and Lpad rows per (item, channel group).  `sched` points to two device ints, zero before the
+// launch (the kernel leaves them zero when it completes): the dynamic tile scheduler's state.
 int launch_amp_gemm_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int m, int half,
                        const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
-                       cudaStream_t s, int* err);
-int launch_conv_pre_tc(const ConvParams& p, const TcStageWeights& w, cudaStream_t s, int* err);
-int launch_convT_tc(const ConvTParams& q, const TcStageWeights& w, cudaStream_t s, int* err);
+                       cudaStream_t s, int* err, int* sched);
 
 // conv_pre and the upsamplers on the persistent GEMM, reading their input as pre-split rows
 // (launch_split_rows) with pad_l zero rows before the sequence and Lpad rows per channel group.
 int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                         int pad_l, long long Lpad, cudaStream_t s, int* err);
+                         int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched);
 int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                      int pad_l, long long Lpad, cudaStream_t s, int* err);
+                      int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched);
 
 }  // namespace mh3a
