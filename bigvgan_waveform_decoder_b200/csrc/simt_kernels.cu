@@ -18,6 +18,7 @@
 // k_convT_simt: transposed conv (upsampling stage) in polyphase form: output t = r*u + phi
 // only meets taps j = (phi + pad) mod r + r*m, so no zero is ever inserted or multiplied.
 #include "mh3a_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace mh3a {
 namespace {
@@ -455,10 +456,10 @@ int launch_convT_simt(const ConvTParams& p, bool mean3, cudaStream_t s) {
 }
 
 // Pointwise (k = 1) conv with few input channels (dec_in_proj, 32 -> 2048): one thread per time
-// sample holds the Cin inputs in registers and sweeps 64 output channels whose weights sit in
+// sample holds the Cin inputs in registers and sweeps 16 output channels whose weights sit in
 // shared memory (every lane reads the same weight: a broadcast).
 constexpr int kPwCin = 64;
-constexpr int kPwOut = 64;
+constexpr int kPwOut = 16;
 constexpr int kPwThreads = 128;
 
 __global__ void __launch_bounds__(kPwThreads) k_conv1x1(const ConvParams p) {
@@ -469,10 +470,14 @@ __global__ void __launch_bounds__(kPwThreads) k_conv1x1(const ConvParams p) {
     const int b = blockIdx.x / tiles;
     const int t = (blockIdx.x % tiles) * kPwThreads + threadIdx.x;
     const int o0 = blockIdx.y * kPwOut;
+    // weights [Cin, 1, Cout]: every copy in flight at once
     for (int i = threadIdx.x; i < Cin * kPwOut; i += kPwThreads) {
         const int c = i / kPwOut, o = i % kPwOut;
-        ws[c][o] = (o0 + o < Cout) ? __ldg(J.w + (size_t)c * Cout + o0 + o) : 0.f;   // [Cin, 1, Cout]
+        if (o0 + o < Cout) ptx::cp_async4(&ws[c][o], J.w + (size_t)c * Cout + o0 + o);
+        else ws[c][o] = 0.f;
     }
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
     __syncthreads();
     if (t >= L) return;
     float z[kPwCin];

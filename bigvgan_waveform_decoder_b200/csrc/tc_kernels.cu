@@ -92,6 +92,14 @@ struct TcPlan {
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
+// Narrow output tiles (NT <= 64) of plain convs take the two-MMA form of the 3xBF16 K-step:
+//   D[0, 2 NT) += A_h [B_h | B_l]      (head x head and head x tail side by side in N)
+//   D[NT, 2 NT) += A_l B_h             (tail x head into the cross columns)
+// so the activation operand is read twice per K-step instead of three times (the MMA of a
+// narrow tile is bound by reading that operand from shared memory).  Their weight blocks store
+// each core column's head rows directly followed by its tail rows.
+__host__ __device__ constexpr bool interleaved_b(int NT, int R) { return R == 1 && NT <= 64; }
+
 __device__ __forceinline__ int floordiv(int a, int r) { return (a >= 0) ? a / r : -((-a + r - 1) / r); }
 
 // sin^2(alpha u) for the tensor-core path: Cody-Waite reduction modulo pi, then the hardware
@@ -217,13 +225,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
                     int shift, phase;
                     bool first;
                     tap_geometry<MODE>(tap, dil, pad, r, p.lo, shift, phase, first);
+                    // weight blocks: [part][core col][row] or, for narrow plain tiles,
+                    // [core col][part][row] (interleaved_b)
+                    constexpr bool ILV = MODE == MODE_AMP && interleaved_b(NT, 1);
+                    constexpr uint32_t b_lbo = (ILV ? 2 * NT : NT) * 16;
                     const uint32_t b_hi = b_smem + sb * pl.SB;
-                    const uint32_t b_lo = b_hi + KG * NT * 16;
+                    const uint32_t b_lo = ILV ? b_hi + NT * 16 : b_hi + KG * NT * 16;
 #pragma unroll
                     for (int kk = 0; kk < KG / 2; ++kk) {
-                        const uint32_t boff = (uint32_t)(2 * kk) * NT * 16;
-                        const uint64_t bh = ptx::smem_desc(b_hi + boff, NT * 16, 128);
-                        const uint64_t bl = ptx::smem_desc(b_lo + boff, NT * 16, 128);
+                        const uint32_t boff = (uint32_t)(2 * kk) * (b_lbo);
+                        const uint64_t bh = ptx::smem_desc(b_hi + boff, b_lbo, 128);
+                        const uint64_t bl = ptx::smem_desc(b_lo + boff, b_lbo, 128);
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + shift) * 16;
@@ -532,6 +544,7 @@ struct GemmParams {
 constexpr int ps_threads(int EW) { return 64 + 32 * EW; }
 constexpr int PS_MAXS = 8;                              // ring stages (max)
 constexpr int PS_TQ = 16;                               // tile-index queue entries
+constexpr int PS_BAR_BYTES = 8 * (4 * PS_MAXS + 5 + PS_TQ) + 8 + 4 * PS_TQ;   // barriers, flags, queue
 constexpr int PS_BUFCOLS = 256;                         // TMEM columns per accumulator buffer
 
 struct PsPlan {
@@ -579,7 +592,9 @@ __device__ __forceinline__ PsTile ps_tile(const GemmParams& p, const PsSched& sc
 template <int MT, int NT, int KGT, int EW, int R>
 __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    static_assert(R * MT * NT <= PS_BUFCOLS, "one accumulator buffer holds R x MT x NT columns");
+    constexpr bool ILV = interleaved_b(NT, R);            // two-MMA K-steps, head | cross columns
+    constexpr int RSTR = ILV ? 2 * NT : R * NT;            // accumulator columns per M tile
+    static_assert(MT * RSTR <= PS_BUFCOLS, "one accumulator buffer holds MT x RSTR columns");
     static_assert(R == 1 || KGT >= 2, "the upsampler uses 16- or 32-channel chunks");
     static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
     static_assert(EW == 8 || EW == 16, "epilogue warps");
@@ -607,6 +622,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_full + PS_TQ);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* tile_q = abort_flag + 1;               // [PS_TQ] tile indices, -1 = no more
+    float* bias_s = reinterpret_cast<float*>(smem + pl.offBar + PS_BAR_BYTES);   // [EW][CW] per warp
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nsa; ++s) {
@@ -642,6 +658,8 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         // Descriptors are built once per ring slot and advanced by adding 16-byte offsets to
         // their low word (the start-address field).
         constexpr uint32_t idesc = ptx::idesc_bf16(128, NT);
+        constexpr uint32_t idesc_2n = ptx::idesc_bf16(128, ILV ? 2 * NT : NT);
+        constexpr uint32_t b_lbo = (ILV ? 2 * NT : NT) * 16;   // bytes between core columns
         constexpr int KK = (KGT == 1) ? 1 : KGT / 2;   // K-steps per tap unit
         const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
         bool ok = *abort_flag == 0;
@@ -670,7 +688,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     if (ucopy == 0) {
                         if (!__all_sync(0xffffffffu, ptx::mbar_wait(&b_full[sb], pb, kWaitLimit))) { ok = false; break; }
                         ptx::tc_fence_after();
-                        bh0 = ptx::desc_lo(b_smem + sb * pl.SB, NT * 16);
+                        bh0 = ptx::desc_lo(b_smem + sb * pl.SB, b_lbo);
                     }
                     if (upass == 0) {
                         if (!__all_sync(0xffffffffu, ptx::mbar_wait(&acc_empty[buf], pacc ^ 1, kWaitLimit))) { ok = false; break; }
@@ -689,14 +707,23 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     }
 #pragma unroll
                     for (int kk = 0; kk < KK; ++kk) {
-                        const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
-                        const uint32_t blk = bhk + (uint32_t)(BG * NT);
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const uint32_t a = ah0 + arow + (uint32_t)(2 * kk * RS + mt * 128);
-                            ptx::mma3_bf16_elect(dbase + (uint32_t)(mt * R * NT), ptx::desc64(a),
-                                                 ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bhk),
-                                                 ptx::desc64(blk), idesc, (first && kk == 0) ? 0u : 1u);
+                            const uint32_t d = dbase + (uint32_t)(mt * RSTR);
+                            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                            if (ILV) {
+                                // core columns 2kk, 2kk+1 hold [heads | tails] of NT rows each
+                                const uint32_t bk = bh + (uint32_t)(2 * kk * 2 * NT);
+                                ptx::mma2_bf16_elect(d, d + (uint32_t)NT, ptx::desc64(a),
+                                                     ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bk), idesc_2n,
+                                                     idesc, acc);
+                            } else {
+                                const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
+                                const uint32_t blk = bhk + (uint32_t)(BG * NT);
+                                ptx::mma3_bf16_elect(d, ptx::desc64(a), ptx::desc64(a + (uint32_t)(KGT * RS)),
+                                                     ptx::desc64(bhk), ptx::desc64(blk), idesc, acc);
+                            }
                         }
                     }
                     ++ucopy;
@@ -804,7 +831,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         const int col0 = (e >> 2) * CW;        // first channel column of this warp ([mt][NT] order)
         const int mt = col0 / NT, oc0 = col0 % NT;
         // regions [mt][phase][NT]: this warp's columns of phase phi start at + phi * NT
-        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(mt * R * NT + oc0);
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(mt * RSTR + oc0);
         constexpr bool kPrefetch = (R == 1) && CW <= 16;   // residual loaded ahead of the MMAs
         const long long Lout = (long long)L * R;
         bool ok = *abort_flag == 0;
@@ -823,6 +850,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             const int t = T.t0 + mt * 128 + q4 * 32 + lane;   // the row (input sample when R > 1)
             const int o_base = T.ot * NT + oc0;
             const long long idx0 = ((long long)T.b * Cout + o_base) * Lout + (long long)R * t;
+            // this warp's bias values, staged in shared memory while the tile's MMAs run (read
+            // back as broadcasts by the final stores)
+            float* bsl = bias_s + (warp - 2) * CW;
+            for (int c = lane; c < CW; c += 32) bsl[c] = (o_base + c < Cout) ? __ldg(J.bias + o_base + c) : 0.f;
+            __syncwarp();
             float res[kPrefetch ? CW : 1];
             if (kPrefetch) {
 #pragma unroll
@@ -842,6 +874,12 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     for (int cb = 0; cb < CW; cb += 16) {
                         float v[16];
                         ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
+                        if (ILV) {
+                            float x[16];
+                            ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + NT + cb), x);
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) v[c] += x[c];
+                        }
 #pragma unroll
                         for (int c = 0; c < 16; ++c) acc[ph * CW + cb + c] += v[c];
                     }
@@ -855,27 +893,30 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                 break;
             }
             if (t < L) {
-                // FC channels at a time: all loads of a group are in flight before its stores
+                // FC channels at a time: all residual loads of a group are in flight before its
+                // stores
                 constexpr int FC = (R * CW > 64) ? 8 : 16;
+                const bool has_res = R == 1 && J.res != nullptr;
 #pragma unroll
                 for (int cb = 0; cb < CW; cb += FC) {
-                    float bs[FC], rs[FC];
+                    float rs[FC];
 #pragma unroll
                     for (int c = 0; c < FC; ++c) {
                         const int o = o_base + cb + c;   // channels past Cout pad the tile
-                        bs[c] = (o < Cout) ? __ldg(J.bias + o) : 0.f;
                         if (kPrefetch) rs[c] = res[cb + c];
-                        else rs[c] = (R == 1 && J.res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * Lout] : 0.f;
+                        else rs[c] = (has_res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * Lout] : 0.f;
                     }
 #pragma unroll
                     for (int c = 0; c < FC; ++c) {
                         if (o_base + cb + c >= Cout) continue;
+                        const float bb = bsl[cb + c];
 #pragma unroll
                         for (int ph = 0; ph < R; ++ph)
-                            J.out[idx0 + (long long)(cb + c) * Lout + ph] = (acc[ph * CW + cb + c] + bs[c]) + rs[c];
+                            J.out[idx0 + (long long)(cb + c) * Lout + ph] = (acc[ph * CW + cb + c] + bb) + rs[c];
                     }
                 }
             }
+            __syncwarp();   // the bias slice is rewritten for the next tile
         }
         if (!ok) {
             *abort_flag = 1;
@@ -1027,7 +1068,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     pl.RS = 128 * MT + span;
     pl.SA = 2 * KGT * pl.RS * 16;
     pl.SB = p.tpu * TAPB;
-    constexpr int kBarBytes = 8 * (4 * PS_MAXS + 5 + PS_TQ) + 8 + 4 * PS_TQ;
+    constexpr int kBarBytes = PS_BAR_BYTES + 4 * EW * 4 * MT * NT / EW;   // + the epilogue's bias slices
     constexpr int kBudget = 227 * 1024 - kBarBytes - 64;
     pl.nsa = (4 * pl.SA <= kBudget / 2) ? 4 : 3;
     if (pl.nsa * pl.SA + 2 * pl.SB > kBudget) pl.nsa = 2;
@@ -1082,7 +1123,7 @@ void amp_layout(int C, int* NT, int* KGT) {
 // columns are the chunk's channel groups; for KGT == 1 a unit is a tap pair and the two core
 // columns are its taps (zero past the last tap).  Rows o >= Cout are zero.
 template <class W>
-void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, TcConv* out) {
+void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, bool interleave, TcConv* out) {
     const int kc = 8 * KGT;
     const int ntiles = (Cout + NT - 1) / NT, nchunks = Cin / kc;
     const int KU = (KGT == 1) ? (K + 1) / 2 : K;
@@ -1090,13 +1131,17 @@ void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, TcConv* out) {
     const size_t n = (size_t)ntiles * nchunks * KU * 2 * BG * NT * 8;  // bf16 elements
     std::vector<uint16_t> buf(n);
     size_t pos = 0;
+    // interleave: [core col][part] (the head rows of a core column directly followed by its tail
+    // rows); otherwise [part][core col]
     for (int ot = 0; ot < ntiles; ++ot)
         for (int chk = 0; chk < nchunks; ++chk)
             for (int unit = 0; unit < KU; ++unit)
-                for (int part = 0; part < 2; ++part)
-                    for (int col = 0; col < BG; ++col)
+                for (int outer = 0; outer < (interleave ? BG : 2); ++outer)
+                    for (int inner = 0; inner < (interleave ? 2 : BG); ++inner)
                         for (int o = 0; o < NT; ++o)
                             for (int e = 0; e < 8; ++e) {
+                                const int part = interleave ? inner : outer;
+                                const int col = interleave ? outer : inner;
                                 const int oo = ot * NT + o;
                                 const int tap = (KGT == 1) ? 2 * unit + col : unit;
                                 const int cc = chk * kc + ((KGT == 1) ? 0 : col * 8) + e;
@@ -1158,17 +1203,19 @@ bool tc_convt_supported(int Cin, int Cout, int r, int K) {
 void prepare_tc_conv(const std::vector<float>& w, int C, int k, TcConv* out) {
     int NT, KGT;
     amp_layout(C, &NT, &KGT);
-    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * C + c) * k + tap]; }, C, C, k, NT, KGT, out);
+    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * C + c) * k + tap]; }, C, C, k, NT, KGT,
+                interleaved_b(NT, 1), out);
 }
 
 void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWeights* out) {
     pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + c) * k + tap]; }, O, I, k, ntile_pre(O), KG,
+                interleaved_b(ntile_pre(O), 1),
                 &out->pre);
 }
 
 void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
     pack_blocks([&](int o, int c, int tap) { return w_iok[((size_t)c * Cout + o) * K + tap]; }, Cout, Cin, K,
-                ntile_convt(Cout, r), kgt_convt(Cin), out);
+                ntile_convt(Cout, r), kgt_convt(Cin), interleaved_b(ntile_convt(Cout, r), r), out);
 }
 
 void tc_finalize(TcStageWeights* w) {

@@ -146,6 +146,24 @@ __device__ __forceinline__ void mma3_bf16_elect(uint32_t d_tmem, uint64_t ah, ui
         : "memory");
 }
 
+// The two-MMA form of a 3xBF16 K-step (one elected lane of a converged warp): `b` describes
+// NT head rows directly followed by NT tail rows, so D[0, 2NT) (+)= Ah [Bh | Bl] under
+// `idesc_2n`, then D[NT, 2NT) += Al Bh under `idesc_n` (same descriptor, first NT rows);
+// `d_cross` = d_tmem + NT.
+__device__ __forceinline__ void mma2_bf16_elect(uint32_t d_tmem, uint32_t d_cross, uint64_t ah, uint64_t al,
+                                                uint64_t b, uint32_t idesc_2n, uint32_t idesc_n,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, q;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %7, 0;\n\t"
+        "setp.eq.b32 q, %7, %7;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %4, %5, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], %3, %4, %6, q;\n\t}" ::"r"(d_tmem),
+        "r"(d_cross), "l"(ah), "l"(al), "l"(b), "r"(idesc_2n), "r"(idesc_n), "r"(accumulate)
+        : "memory");
+}
+
 // tcgen05.commit by one elected lane of a converged warp.
 __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
     asm volatile(
