@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 
 #include "act_kernels.cuh"
+#include "act_math.cuh"
 #include "tc_ptx.cuh"
 
 namespace mh3a {
@@ -31,7 +32,6 @@ namespace {
 constexpr int TT = 512;                   // output rows per block
 constexpr int RUN = 16;                   // outputs per lane (TT = 32 RUN)
 constexpr int NT_ACT = 256;               // threads per block (8 warps: one per channel)
-constexpr int NS = 2 * RUN + 10;          // SnakeBeta values one lane's decimation reads
 // Shared layout: per channel a window of x and a row of outputs, each with 4 floats
 // of padding after every 16 so that lanes reading 16-float runs hit distinct banks.
 constexpr int XF = TT + 16;               // x[t0 - 8, t0 + TT + 8)
@@ -39,63 +39,9 @@ constexpr int XF_P = XF + XF / 16 * 4;
 constexpr int TF_P = TT + TT / 16 * 4;
 constexpr int SMEM_FLOATS = 8 * (XF_P + TF_P);
 
-__device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
-__device__ __forceinline__ int skew(int i) { return i + ((i >> 4) << 2); }
-
-// sin^2(alpha u): Cody-Waite reduction modulo pi, then the hardware sine on [-pi/2, pi/2]
-// (absolute error near 2^-21, far below the 3xBF16 operand error).
-// The nearest integer k = rint(v / pi) is formed by adding and subtracting 1.5 * 2^23 in
-// round-to-nearest fp32 arithmetic, exact for |v / pi| < 2^22.
-__device__ __forceinline__ float sin_sq_fast(float alpha, float u) {
-    const float kInvPi = 0.318309886183790671538f;
-    const float kPiHi = 3.14159274101257324219f;
-    const float kPiLo = -8.74227800037248297e-08f;
-    const float kRound = 12582912.0f;  // 1.5 * 2^23
-    const float v = alpha * u;
-    const float k = __fsub_rn(__fmaf_rn(v, kInvPi, kRound), kRound);
-    float r = fmaf(-k, kPiHi, v);
-    r = fmaf(-k, kPiLo, r);
-    const float s = __sinf(r);
-    return s * s;
-}
-
-// Two fp32 values -> packed bf16x2 (round to nearest even), first value in the low half.
-__device__ __forceinline__ uint32_t pack2(float first, float second) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(first, second);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// Head/tail split of two values: heads packed in *h, tails (v - head) packed in *l.
-__device__ __forceinline__ void split2(float a, float b, uint32_t* h, uint32_t* l) {
-    const uint32_t hp = pack2(a, b);
-    const float ha = __uint_as_float(hp << 16), hb = __uint_as_float(hp & 0xFFFF0000u);
-    *h = hp;
-    *l = pack2(a - ha, b - hb);
-}
-
-
-// SnakeBeta value j of a lane's window, n = 2 (t0 + q0) - 5 + j, from xv[k] = x[t0 + q0 - 8 + k]
-// (j even: odd phase n = 2m + 1; j odd: even phase n = 2m).
-template <int J>
-__device__ __forceinline__ float snake_at(const ActFilter& f, const float* xv, float al, float ib) {
-    float u = 0.f;
-    if (J % 2 == 0) {
-#pragma unroll
-        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k], xv[8 + J / 2 - k], u);
-    } else {
-#pragma unroll
-        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k + 1], xv[8 + (J - 1) / 2 - k], u);
-    }
-    return fmaf(sin_sq_fast(al, u), ib, u);
-}
-
-template <int J0, int J1>
-__device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv, float al, float ib, float* s) {
-    if constexpr (J0 < J1) {
-        s[J0] = snake_at<J0>(f, xv, al, ib);
-        snake_range<J0 + 1, J1>(f, xv, al, ib, s);
-    }
-}
+using actm::clampi;
+using actm::skew;
+using actm::split2;
 
 // One tile: rows [t0, t0 + TT).  EDGE = false requires 8 <= t0 and t0 + TT + 8 <= L, so that
 // neither the input window nor the 2x-rate SnakeBeta window reaches past a sequence end.  EDGE
@@ -129,58 +75,8 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
     __syncwarp();
     const float al = __ldg(J.alpha + g * 8 + c), ib = __ldg(J.inv_beta + g * 8 + c);
     const int q0 = RUN * lane;
-    float xv[32];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float4 v = *reinterpret_cast<const float4*>(xs + skew(q0 + 4 * k));
-        xv[4 * k] = v.x;
-        xv[4 * k + 1] = v.y;
-        xv[4 * k + 2] = v.z;
-        xv[4 * k + 3] = v.w;
-    }
-    float s[NS];
-    snake_range<5, 5 + 2 * RUN>(p.filt, xv, al, ib, s);     // the lane's own 2 RUN values
-    // The 5 values left of lane 0's run and right of lane 31's run: lanes 0-4 and 5-9 form one
-    // each (value j of lane 0's window, resp. j = 37 .. 41 of lane 31's), from the same taps.
-    float hv = 0.f;
-    if (lane < 10) {
-        const int j = (lane < 5) ? lane : lane + 2 * RUN;
-        const int i0 = ((lane < 5) ? 0 : RUN * 31) + 8 + (j >> 1);
-        const int par = j & 1;
-        float u = 0.f;
-#pragma unroll
-        for (int k = 0; k < 6; ++k) u = fmaf(p.filt.up[2 * k + par], xs[skew(i0 - k)], u);
-        hv = fmaf(sin_sq_fast(al, u), ib, u);
-    }
-#pragma unroll
-    for (int j = 0; j < 5; ++j) {
-        const float from_left = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
-        const float from_right = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
-        const float h = __shfl_sync(0xffffffffu, hv, (lane == 31) ? j + 5 : j);
-        s[j] = (lane == 0) ? h : from_left;
-        s[j + 5 + 2 * RUN] = (lane == 31) ? h : from_right;
-    }
-    if (EDGE) {
-        // replicate padding at the 2x rate: n < 0 takes s(0), n > 2L - 1 takes s(2L - 1)
-        const int n0 = 2 * (t0 + q0) - 5;
-        const int j0 = -n0, je = 2 * L - 1 - n0;
-        float sf = s[0], sl = s[NS - 1];
-#pragma unroll
-        for (int j = 0; j < NS; ++j) {
-            sf = (j == j0) ? s[j] : sf;
-            sl = (j == je) ? s[j] : sl;
-        }
-#pragma unroll
-        for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
-    }
     float a[RUN];
-#pragma unroll
-    for (int i = 0; i < RUN; ++i) {
-        float v = 0.f;
-#pragma unroll
-        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(p.filt.down[j], s[2 * i + j], v);
-        a[i] = v;
-    }
+    actm::act_lane<RUN, EDGE>(p.filt, xs, al, ib, t0, L, a);
     float* trow = T + c * TF_P;
 #pragma unroll
     for (int k = 0; k < RUN / 4; ++k)

@@ -1,0 +1,160 @@
+// act_math.cuh -- the anti-aliased SnakeBeta of one channel, register-blocked per lane, shared by
+// the standalone activation kernel and the producer warps of the fused tensor-core GEMM.
+//
+//   a = down2(snake(up2(x)))      (FastVideo "minimax_h3_audio_vae" page, `_activation1d`;
+//                                  filter from `kaiser_sinc_filter1d`)
+// up2: replicate-pad 5, stride-2 transposed conv with the 12 taps at gain 2, crop 15 per side;
+// in polyphase form u[2m] = sum_q 2 f[2q+1] x[m+2-q], u[2m+1] = sum_q 2 f[2q] x[m+3-q];
+// snake: s = u + sin^2(alpha u) / (beta + 1e-9); down2: a[t] = sum_j f[j] s[2t+j-5] with s
+// replicate-padded (index clamped to [0, 2L)).
+//
+// A warp computes 32 RUN consecutive outputs of one channel, rows [tw, tw + 32 RUN): lane l owns
+// rows tw + RUN l + [0, RUN).  It forms the 2 RUN SnakeBeta values at the 2x rate that belong to
+// its rows in registers, receives the 5 + 5 halo values from its neighbour lanes by warp
+// shuffles (the two values outside the warp's run come from lanes 0-9, one each), and decimates
+// in registers.  The input window x[tw - 8, tw + 32 RUN + 8) sits in shared memory with 4 floats
+// of padding after every 16 (skew), so that lanes reading their runs hit distinct banks.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "mh3a_internal.cuh"
+
+namespace mh3a {
+namespace actm {
+
+__device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+__device__ __forceinline__ int skew(int i) { return i + ((i >> 4) << 2); }
+// skewed size of a window of n floats
+__host__ __device__ constexpr int skewed(int n) { return n + n / 16 * 4 + 4; }
+
+// sin^2(alpha u): Cody-Waite reduction modulo pi, then the hardware sine on [-pi/2, pi/2]
+// (absolute error near 2^-21, far below the 3xBF16 operand error).
+// The nearest integer k = rint(v / pi) is formed by adding and subtracting 1.5 * 2^23 in
+// round-to-nearest fp32 arithmetic, exact for |v / pi| < 2^22.
+__device__ __forceinline__ float sin_sq_fast(float alpha, float u) {
+    const float kInvPi = 0.318309886183790671538f;
+    const float kPiHi = 3.14159274101257324219f;
+    const float kPiLo = -8.74227800037248297e-08f;
+    const float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float v = alpha * u;
+    const float k = __fsub_rn(__fmaf_rn(v, kInvPi, kRound), kRound);
+    float r = fmaf(-k, kPiHi, v);
+    r = fmaf(-k, kPiLo, r);
+    const float s = __sinf(r);
+    return s * s;
+}
+
+// Two fp32 values -> packed bf16x2 (round to nearest even), first value in the low half.
+__device__ __forceinline__ uint32_t pack2(float first, float second) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(first, second);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Head/tail split of two values: heads packed in *h, tails (v - head) packed in *l.
+__device__ __forceinline__ void split2(float a, float b, uint32_t* h, uint32_t* l) {
+    const uint32_t hp = pack2(a, b);
+    const float ha = __uint_as_float(hp << 16), hb = __uint_as_float(hp & 0xFFFF0000u);
+    *h = hp;
+    *l = pack2(a - ha, b - hb);
+}
+
+// SnakeBeta value j of a lane's window, n = 2 (tw + q0) - 5 + j, from xv[k] = x[tw + q0 - 8 + k]
+// (j even: odd phase n = 2m + 1; j odd: even phase n = 2m).
+template <int J>
+__device__ __forceinline__ float snake_at(const ActFilter& f, const float* xv, float al, float ib) {
+    float u = 0.f;
+    if (J % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k], xv[8 + J / 2 - k], u);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k + 1], xv[8 + (J - 1) / 2 - k], u);
+    }
+    return fmaf(sin_sq_fast(al, u), ib, u);
+}
+
+template <int J0, int J1>
+__device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv, float al, float ib, float* s) {
+    if constexpr (J0 < J1) {
+        s[J0] = snake_at<J0>(f, xv, al, ib);
+        snake_range<J0 + 1, J1>(f, xv, al, ib, s);
+    }
+}
+
+// Outputs a[k] = act(x)[tw + RUN lane + k] of one channel (RUN even).  xs: the skewed window,
+// logical index i <-> x[tw - 8 + i], at least 32 RUN + 16 floats, staged with the sequence's
+// replicate padding when EDGE.  EDGE also substitutes the end values for SnakeBeta positions
+// outside [0, 2L); rows outside [0, L) are the caller's to discard.  Called by all 32 lanes.
+template <int RUN, bool EDGE>
+__device__ __forceinline__ void act_lane(const ActFilter& f, const float* xs, float al, float ib, int tw, int L,
+                                         float (&a)[RUN]) {
+    static_assert(RUN % 2 == 0, "lane runs start on 8-byte boundaries");
+    constexpr int NS = 2 * RUN + 10;                          // SnakeBeta values a lane reads
+    constexpr int NXV = (RUN % 4 == 0) ? (RUN + 11 + 3) / 4 * 4 : (RUN + 11 + 1) / 2 * 2;
+    const int lane = threadIdx.x & 31;
+    const int q0 = RUN * lane;
+    float xv[NXV];
+    if constexpr (RUN % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < NXV / 4; ++k) {
+            const float4 v = *reinterpret_cast<const float4*>(xs + skew(q0 + 4 * k));
+            xv[4 * k] = v.x;
+            xv[4 * k + 1] = v.y;
+            xv[4 * k + 2] = v.z;
+            xv[4 * k + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NXV / 2; ++k) {
+            const float2 v = *reinterpret_cast<const float2*>(xs + skew(q0 + 2 * k));
+            xv[2 * k] = v.x;
+            xv[2 * k + 1] = v.y;
+        }
+    }
+    float s[NS];
+    snake_range<5, 5 + 2 * RUN>(f, xv, al, ib, s);     // the lane's own 2 RUN values
+    // The 5 values left of lane 0's run and right of lane 31's run: lanes 0-4 and 5-9 form one
+    // each (value j of lane 0's window, resp. j = 2 RUN + 5 .. 2 RUN + 9 of lane 31's).
+    float hv = 0.f;
+    if (lane < 10) {
+        const int j = (lane < 5) ? lane : lane + 2 * RUN;
+        const int i0 = ((lane < 5) ? 0 : RUN * 31) + 8 + (j >> 1);
+        const int par = j & 1;
+        float u = 0.f;
+#pragma unroll
+        for (int k = 0; k < 6; ++k) u = fmaf(f.up[2 * k + par], xs[skew(i0 - k)], u);
+        hv = fmaf(sin_sq_fast(al, u), ib, u);
+    }
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+        const float from_left = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
+        const float from_right = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
+        const float h = __shfl_sync(0xffffffffu, hv, (lane == 31) ? j + 5 : j);
+        s[j] = (lane == 0) ? h : from_left;
+        s[j + 5 + 2 * RUN] = (lane == 31) ? h : from_right;
+    }
+    if (EDGE) {
+        // replicate padding at the 2x rate: n < 0 takes s(0), n > 2L - 1 takes s(2L - 1)
+        const int n0 = 2 * (tw + q0) - 5;
+        const int j0 = -n0, je = 2 * L - 1 - n0;
+        float sf = s[0], sl = s[NS - 1];
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            sf = (j == j0) ? s[j] : sf;
+            sl = (j == je) ? s[j] : sl;
+        }
+#pragma unroll
+        for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
+    }
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(f.down[j], s[2 * i + j], v);
+        a[i] = v;
+    }
+}
+
+}  // namespace actm
+}  // namespace mh3a
