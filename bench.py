@@ -36,6 +36,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decoded audio-seconds/sec at 32 kHz on 1 B200; % of roofline per stage"
+
+# Tile shape <MT, NT, KGT, EW, R> of the persistent GEMM per AMP width (as dispatched by the
+# library), for labelling the roofline's kernel.
+GEMM_TILE = {512: "1, 256, 4, 8, 1", 256: "1, 256, 4, 8, 1", 128: "2, 128, 4, 8, 1",
+             64: "2, 64, 4, 16, 1", 32: "2, 32, 4, 16, 1", 16: "4, 16, 2, 16, 1", 8: "4, 16, 1, 16, 1"}
+# DRAM bytes (read + write) per launch of that GEMM kernel on this workload, keyed by (channels,
+# B * N), from one ncu capture (profiles/k_gemm_ps_stage1_B2_L10000.md); null when unmeasured
+# or when the kernel changed after the capture.
+GEMM_TRAFFIC = {(256, 800): 85.8e6}
 UNIT = "audio-s/s"
 WORKLOAD = 3
 FLUSH_BYTES = 256 << 20
@@ -195,6 +204,13 @@ def run_ours(args):
         flush.fill_(1.0)
         dec.decode(x, out)
     torch.cuda.synchronize()
+    # the dominant AMP stage of the warm-up decodes gets per-launch kernel events while timed
+    warm = dec.segment_times()
+    n_stages = len(arch.rates)
+    amp_ms = [warm[3 + 2 * i] if 3 + 2 * i < len(warm) else 0.0 for i in range(n_stages)]
+    kstage = max(range(n_stages), key=lambda i: amp_ms[i])
+    kstage = kstage if dec.stage_uses_tensor_cores(kstage) else -1
+    dec.set_kernel_profiling(kstage)
     barrier()
     torch.cuda.synchronize()
 
@@ -202,6 +218,7 @@ def run_ours(args):
     clocks.start()
     launches0 = dec.launch_count()
     step_ms, seg_sum = [], None
+    kern_sum = [[0.0, 0.0] for _ in range(n_stages)]   # per AMP stage: activation, GEMM ms
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for k in range(args.steps):
         flush.fill_(float(k))
@@ -212,12 +229,17 @@ def run_ours(args):
         step_ms.append(ev0.elapsed_time(ev1))
         seg = dec.segment_times()
         seg_sum = seg if seg_sum is None else [a + b for a, b in zip(seg_sum, seg)]
+        if kstage >= 0:
+            a_ms, g_ms = dec.stage_kernel_times(kstage)
+            kern_sum[kstage][0] += a_ms
+            kern_sum[kstage][1] += g_ms
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     launches = dec.launch_count() - launches0
     clk = clocks.stop()
     dec.set_profiling(False)
+    dec.set_kernel_profiling(-1)
 
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -266,11 +288,27 @@ def run_ours(args):
     if dom is not None:
         sgm, ms = segs[dom], seg_ms[dom]
         launches_in_seg = 6 if sgm.name.startswith("amp") else 1
-        if sgm.tensor:
+        stage_i = int(sgm.name[3:]) if sgm.name.startswith("amp") else None
+        if sgm.tensor and stage_i is not None and kern_sum[stage_i][1] > 0:
+            # the stage's GEMM kernel alone: algorithmic flops of one launch (3 residual blocks)
+            # over its average launch duration, from the per-launch events of the timed steps
+            gemm_launch_ms = kern_sum[stage_i][1] / args.steps / 6
+            act_launch_ms = kern_sum[stage_i][0] / args.steps / 6
+            achieved = sgm.conv_flops / 6 / (gemm_launch_ms * 1e-3) / 1e12
+            C = arch.decoder_dim >> (stage_i + 1)
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
+                        "frac": achieved / p_tc, "traffic": GEMM_TRAFFIC.get((C, B * N)),
+                        "kernel": f"k_gemm_ps<{GEMM_TILE.get(C, '?')}> ({sgm.name} conv, 3 residual blocks per launch)",
+                        "launch_ms": gemm_launch_ms, "launches_per_step": launches_in_seg,
+                        "flops_per_launch": sgm.conv_flops / 6,
+                        "activation_kernel_ms_per_launch": act_launch_ms,
+                        "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
+                                      "bf16 products per fp32 product"}
+        elif sgm.tensor:
             achieved = sgm.conv_flops / (ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
                         "frac": achieved / p_tc, "traffic": None,
-                        "kernel": f"{sgm.name} conv (3 residual blocks per launch)",
+                        "kernel": f"{sgm.name} conv (segment)",
                         "launches_per_step": launches_in_seg,
                         "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
                                       "bf16 products per fp32 product"}

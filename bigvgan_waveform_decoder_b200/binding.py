@@ -94,6 +94,10 @@ def load():
     L.mh3a_amp_stage.restype = C.c_int
     L.mh3a_set_profiling.argtypes = [vp, C.c_int]
     L.mh3a_set_profiling.restype = C.c_int
+    L.mh3a_set_kernel_profiling.argtypes = [vp, C.c_int]
+    L.mh3a_set_kernel_profiling.restype = C.c_int
+    L.mh3a_stage_kernel_times.argtypes = [vp, C.c_int, C.POINTER(C.c_float), C.POINTER(C.c_float)]
+    L.mh3a_stage_kernel_times.restype = C.c_int
     L.mh3a_segment_times.argtypes = [vp, C.POINTER(C.c_float), C.c_int, C.POINTER(C.c_int)]
     L.mh3a_segment_times.restype = C.c_int
     L.mh3a_launch_count.argtypes = [vp]
@@ -232,6 +236,16 @@ class Decoder:
 
     def set_profiling(self, on: bool):
         _check(load().mh3a_set_profiling(self._h, 1 if on else 0), "mh3a_set_profiling")
+
+    def set_kernel_profiling(self, stage: int):
+        """Events around the activation and GEMM launches of one AMP stage (-1: none)."""
+        _check(load().mh3a_set_kernel_profiling(self._h, stage), "mh3a_set_kernel_profiling")
+
+    def stage_kernel_times(self, stage: int):
+        """(activation ms, GEMM ms) summed over the AMP stage's six layers of the last decode."""
+        a, g = C.c_float(), C.c_float()
+        _check(load().mh3a_stage_kernel_times(self._h, stage, C.byref(a), C.byref(g)), "mh3a_stage_kernel_times")
+        return a.value, g.value
 
     def segment_times(self):
         buf = (C.c_float * 64)()

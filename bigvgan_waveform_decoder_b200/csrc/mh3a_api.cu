@@ -136,6 +136,12 @@ struct mh3a_handle {
     bool profiling = false;
     cudaEvent_t ev[kMaxSegments + 1] = {};
     int nseg = 0;
+    // kernel profiling of one AMP stage: events before the activation, between it and the
+    // GEMM, and after the GEMM of each of its 6 layers
+    int kprof_stage = -1;
+    cudaEvent_t kev[6][3] = {};
+    bool kev_made = false;
+    int kev_rec = -1;                       // the stage the last decode recorded
     long long launches = 0;
 };
 
@@ -336,10 +342,18 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                     ap.job[j].a_hi = h->A_hi[j];
                     ap.job[j].a_lo = h->A_lo[j];
                 }
+                const bool kprof = h->kprof_stage == stage && h->kev_made;
+                const int li = 2 * m + half;
+                if (kprof) CK_CUDA(cudaEventRecord(h->kev[li][0], s), "cudaEventRecord");
                 mh3a_status st = counted(h, launch_act_split(ap, nrb, s));
                 if (st) return st;
+                if (kprof) CK_CUDA(cudaEventRecord(h->kev[li][1], s), "cudaEventRecord");
                 const long long Lpad = (long long)L + kApadL + kApadR;
                 n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err, h->dev_err + 16);
+                if (kprof && n > 0) {
+                    CK_CUDA(cudaEventRecord(h->kev[li][2], s), "cudaEventRecord");
+                    if (li == 5) h->kev_rec = stage;
+                }
             } else {
                 n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             }
@@ -600,6 +614,9 @@ void mh3a_destroy(mh3a_handle* h) {
     cudaDeviceSynchronize();
     for (auto& e : h->ev)
         if (e) cudaEventDestroy(e);
+    for (auto& li : h->kev)
+        for (auto& e : li)
+            if (e) cudaEventDestroy(e);
     if (h->warena) cudaFree(h->warena);
     if (h->arena) cudaFree(h->arena);
     cudaSetDevice(prev);
@@ -812,6 +829,41 @@ mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L, int sta
 mh3a_status mh3a_set_profiling(mh3a_handle* h, int enable) {
     if (!h) return MH3A_ERR_INVALID_ARG;
     h->profiling = enable != 0;
+    return MH3A_OK;
+}
+
+mh3a_status mh3a_set_kernel_profiling(mh3a_handle* h, int stage) {
+    if (!h || stage < -1 || stage >= h->cfg.n_stages) return MH3A_ERR_INVALID_ARG;
+    if (stage >= 0 && !h->kev_made) {
+        int prev = 0;
+        cudaGetDevice(&prev);
+        cudaSetDevice(h->device);
+        cudaError_t e_ = cudaSuccess;
+        for (auto& li : h->kev)
+            for (auto& e : li)
+                if (e_ == cudaSuccess) e_ = cudaEventCreate(&e);
+        cudaSetDevice(prev);
+        if (e_ != cudaSuccess) return cuda_fail(e_, "cudaEventCreate");
+        h->kev_made = true;
+    }
+    h->kprof_stage = stage;
+    h->kev_rec = -1;
+    return MH3A_OK;
+}
+
+mh3a_status mh3a_stage_kernel_times(mh3a_handle* h, int stage, float* act_ms, float* gemm_ms) {
+    if (!h || !act_ms || !gemm_ms || stage < 0 || stage >= h->cfg.n_stages) return MH3A_ERR_INVALID_ARG;
+    *act_ms = 0.f;
+    *gemm_ms = 0.f;
+    if (!h->kev_made || h->kev_rec != stage) return MH3A_ERR_UNSUPPORTED;
+    CK_CUDA(cudaEventSynchronize(h->kev[5][2]), "cudaEventSynchronize");
+    for (int li = 0; li < 6; ++li) {
+        float a = 0.f, g = 0.f;
+        CK_CUDA(cudaEventElapsedTime(&a, h->kev[li][0], h->kev[li][1]), "cudaEventElapsedTime");
+        CK_CUDA(cudaEventElapsedTime(&g, h->kev[li][1], h->kev[li][2]), "cudaEventElapsedTime");
+        *act_ms += a;
+        *gemm_ms += g;
+    }
     return MH3A_OK;
 }
 

@@ -173,6 +173,17 @@ MH3A_API mh3a_status mh3a_amp_stage_static(mh3a_handle* h, const float* x, int B
 MH3A_API mh3a_status mh3a_set_profiling(mh3a_handle* h, int enable);
 MH3A_API mh3a_status mh3a_segment_times(mh3a_handle* h, float* ms, int cap, int* count);
 
+/* Per-kernel device timing of one tensor-core AMP stage.  After
+ * mh3a_set_kernel_profiling(h, stage), each decode records CUDA events around that stage's six
+ * activation launches and six GEMM launches (stage -1: none; each event record costs a few
+ * microseconds of stream time, so only one stage is instrumented).  mh3a_stage_kernel_times
+ * waits for the last decode and writes the summed durations (milliseconds) of the stage's
+ * activation launches to *act_ms and of its GEMM launches to *gemm_ms.  MH3A_ERR_INVALID_ARG
+ * for a NULL argument or an out-of-range stage; MH3A_ERR_UNSUPPORTED if the last decode did not
+ * record that stage (another stage selected, or the stage not on the tensor cores). */
+MH3A_API mh3a_status mh3a_set_kernel_profiling(mh3a_handle* h, int stage);
+MH3A_API mh3a_status mh3a_stage_kernel_times(mh3a_handle* h, int stage, float* act_ms, float* gemm_ms);
+
 /* 1 if the AMP convolutions of `stage` run on the tensor cores for this handle, 0 if on the
  * fp32 CUDA cores, -1 for a NULL handle or an out-of-range stage. */
 MH3A_API int mh3a_stage_uses_tensor_cores(const mh3a_handle* h, int stage);
