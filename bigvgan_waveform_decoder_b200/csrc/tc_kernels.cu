@@ -1,42 +1,35 @@
-// tc_kernels.cu -- tensor-core (tcgen05 / TMEM) convolutions of the decode.
+// tc_kernels.cu -- tensor-core (tcgen05 / TMEM) convolutions of the decode, as implicit GEMMs
+// D[row, o] = sum_k A[row, k] B[o, k] with M = time rows (128-row accumulators in tensor
+// memory), N = output channels and K = input channels x taps.
 //
-// One kernel template, three modes, all implicit GEMMs D[row, o] = sum_k A[row, k] B[o, k]
-// with M = time rows (128-row accumulators in tensor memory, MT of them per CTA), N = output
-// channels (NT per CTA) and K = input channels x taps:
-//
-//  AMP    one conv layer of every residual block of an AMP stage (blockIdx.z = block, the
-//         heaviest kernel first):
-//           y[o, t] = bias[o] + sum_{c, tap} W[o, c, tap] a[c, t + tap*dil - pad] (+ res[o, t])
-//         with a = down2(snake(up2(x))), the anti-aliased SnakeBeta of the FastVideo
-//         "minimax_h3_audio_vae" page's `_activation1d`, computed by the producer warps.
-//  PLAIN  the same conv without the activation (conv_pre: k = 7, padding 3).
-//  CONVT  a weight-normed transposed conv (`ups.i.0`) in polyphase form: output t = r u + phi
-//         only meets taps j = (phi + pad) mod r + r m, and reads input u + (phi + pad - j) / r.
-//         Every tap therefore is a plain shifted-window product over the input rows, so no zero
-//         is ever inserted or multiplied; each phase owns its own accumulators, and the epilogue
-//         writes phase phi of row u to output sample r u + phi.
+//  k_gemm_ps   the persistent GEMM that runs every tensor-core conv of a decode: the AMP
+//              residual-block convs (the anti-aliased SnakeBeta of the FastVideo
+//              "minimax_h3_audio_vae" page's `_activation1d` already written as the A operand
+//              by the activation kernel), conv_pre, and the weight-normed transposed convs
+//              (`ups.i.0`) in polyphase form: output t = r u + phi only meets taps
+//              j = (phi + pad) mod r + r m, which read input u + (phi + pad - j) / r, so no zero
+//              is ever inserted or multiplied.  Its design notes precede the kernel.
+//  k_conv_tc   a fused AMP layer (activation computed by 16 producer warps into the A operand
+//              in shared memory) for the allocation-free stage entry point, which has no
+//              operand arrays.
 //
 // Precision (3xBF16): every fp32 operand is split into a bf16 head h = bf16(v) and a bf16
 // tail l = bf16(v - h); the product is accumulated as A_h B_h + A_h B_l + A_l B_h in fp32.
 //
 // Accumulation: the tensor core rounds its fp32 accumulator toward zero at every instruction,
 // so a long K loop into one accumulator builds a bias of about (instructions) x 2^-24
-// relative.  Each (M tile, phase) therefore owns NACC accumulators of NT columns: head x head
-// products rotate over the first NACC-1 by chunk, and the small cross terms (head x tail,
-// tail x head) go to the last one; the epilogue adds them in fp32 with round-to-nearest.
+// relative.  k_gemm_ps bounds every accumulator to one pass of at most 8 K-steps and adds the
+// passes in fp32 registers with round-to-nearest; k_conv_tc gives each M tile NACC
+// accumulators (head x head products rotating over the first NACC-1 by chunk, the cross terms
+// in the last) and adds them in the epilogue.
 //
 // Shared-memory operands use the no-swizzle K-major canonical layout: core matrices of 8 rows
 // x 16 bytes (8 bf16 along K).  The input window is stored with ALL its rows 16 bytes apart
 // inside each 8-channel group, so the operand of any tap is the same window started a few rows
 // later: only the descriptor start address moves.  Weights are pre-split and pre-laid-out at
-// create time in that layout, one contiguous block per (output tile, 32-channel chunk, tap),
-// so one 1-D bulk copy stages it.
-//
-// Warp roles: warp 0 -- TMEM allocation and the MMA issuer (one thread); warp 1 -- weight bulk
-// copies (one thread); warps 2..17 -- input producers (cp.async prefetch of the next 8-channel
-// window, activation or plain split into the A operand), then the epilogue (TMEM -> registers
-// -> bias + residual -> fp32 stores along time).  Every mbarrier wait is bounded; a timeout
-// raises the error flag, and the kernel drains and returns.
+// create time in that layout, one contiguous block per (output tile, K chunk, tap or tap pair),
+// so 1-D bulk copies stage them.  Every mbarrier wait is bounded; a timeout raises the error
+// flag, and the kernel drains and returns.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -56,12 +49,8 @@ constexpr int NSA = 2;              // activation pipeline depth
 constexpr int NSB = 3;              // weight pipeline depth
 constexpr uint64_t kWaitLimit = 1000000000ull;  // ns; legitimate waits last milliseconds
 
-enum Mode : int { MODE_AMP = 0, MODE_PLAIN = 1, MODE_CONVT = 2 };
-
 struct TcJob {
-    const float* x0;
-    const float* x1;     // with x2: the input is (x0 + x1 + x2) / 3 (CONVT after an AMP stage)
-    const float* x2;
+    const float* x0;     // the layer input [B, Cin, L]
     const uint16_t* w;   // pre-split operand blocks
     const float* bias;
     const float* alpha;
@@ -74,10 +63,8 @@ struct TcJob {
 struct TcParams {
     TcJob job[MH3A_MAX_RESBLOCKS];
     int Cin, Cout;
-    int L;               // input length (= output length except CONVT: output r * L)
+    int L;               // sequence length (input = output)
     int B, tiles_t;
-    int r;               // CONVT rate (1 otherwise)
-    int lo;              // CONVT: window rows before the tile (the largest negative tap shift)
     ActFilter filt;
     int* err;
 };
@@ -99,8 +86,6 @@ __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? l
 // narrow tile is bound by reading that operand from shared memory).  Their weight blocks store
 // each core column's head rows directly followed by its tail rows.
 __host__ __device__ constexpr bool interleaved_b(int NT, int R) { return R == 1 && NT <= 64; }
-
-__device__ __forceinline__ int floordiv(int a, int r) { return (a >= 0) ? a / r : -((-a + r - 1) / r); }
 
 // sin^2(alpha u) for the tensor-core path: Cody-Waite reduction modulo pi, then the hardware
 // sine on [-pi/2, pi/2] (absolute error near 2^-21, far below the 3xBF16 operand error).
@@ -126,29 +111,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
 
 __device__ __forceinline__ float bf16_round(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-// Row shift (in window rows) and phase of tap j.
-template <int MODE>
-__device__ __forceinline__ void tap_geometry(int j, int dil, int pad, int r, int lo, int& shift, int& phase,
-                                             bool& first) {
-    if (MODE == MODE_CONVT) {
-        phase = ((j - pad) % r + r) % r;
-        shift = floordiv(phase + pad - j, r) + lo;
-        first = j == (phase + pad) % r;   // the smallest tap of this phase
-    } else {
-        phase = 0;
-        shift = j * dil;
-        first = j == 0;
-    }
-}
-
-template <int MODE, int MT, int NT, int NACC, int R>
+// Fused AMP layer.  Warp roles: warp 0 -- TMEM allocation and the MMA issuer (one thread);
+// warp 1 -- weight bulk copies (one thread); warps 2..17 -- input producers (cp.async prefetch
+// of the next 8-channel window, SnakeBeta at the 2x rate, decimation into the A operand), then
+// the epilogue (TMEM -> registers -> bias + residual -> fp32 stores along time).
+template <int MT, int NT, int NACC>
 __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const TcPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int NHH = NACC - 1;
-    constexpr int USED = MT * R * NT * NACC;
+    constexpr int USED = MT * NT * NACC;
     static_assert(NACC >= 2 && USED <= 512, "tensor memory holds 512 columns");
     constexpr int NCOLS = (USED <= 32) ? 32 : (USED <= 64) ? 64 : (USED <= 128) ? 128 : (USED <= 256) ? 256 : 512;
-    constexpr int NIN = (MODE == MODE_CONVT) ? 3 : 1;   // staged input buffers (CONVT may average 3)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TcJob& J = p.job[blockIdx.z];
     const int K = J.K, dil = J.dil, pad = J.pad;
@@ -158,16 +131,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
     const int o_tile = blockIdx.y;
     const int o0 = o_tile * NT;
     const int nchunks = Cin / KC;
-    const int span = (MODE == MODE_CONVT) ? (pl.RS - 128 * MT) : (K - 1) * dil;
+    const int span = (K - 1) * dil;
     const int ROWS = 128 * MT + span;
     const int RS = pl.RS;
-    const int r = (MODE == MODE_CONVT) ? p.r : 1;
-    const bool mean3 = (MODE == MODE_CONVT) && J.x1 != nullptr;
 
     uint8_t* As = smem;                        // [NSA][2][KG][RS][16 B]
     uint8_t* Bs = smem + pl.offB;              // [NSB][2][KG][NT][16 B]
-    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [2][NIN][8][XWs] (double buffer)
-    float* sw = xs + 2 * NIN * 8 * pl.XWs;                  // [8][SWs] (AMP only)
+    float* xs = reinterpret_cast<float*>(smem + pl.offX);  // [2][8][XWs] (double buffer)
+    float* sw = xs + 2 * 8 * pl.XWs;                        // [8][SWs] SnakeBeta rows
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pl.offBar);
     uint64_t* a_full = bars;
     uint64_t* a_empty = bars + NSA;
@@ -222,12 +193,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
                     const int sb = u % NSB;
                     if (!ptx::mbar_wait(&b_full[sb], (u / NSB) & 1, kWaitLimit)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    int shift, phase;
-                    bool first;
-                    tap_geometry<MODE>(tap, dil, pad, r, p.lo, shift, phase, first);
-                    // weight blocks: [part][core col][row] or, for narrow plain tiles,
+                    const int shift = tap * dil;
+                    const bool first = tap == 0;
+                    // weight blocks: [part][core col][row] or, for narrow tiles,
                     // [core col][part][row] (interleaved_b)
-                    constexpr bool ILV = MODE == MODE_AMP && interleaved_b(NT, 1);
+                    constexpr bool ILV = interleaved_b(NT, 1);
                     constexpr uint32_t b_lbo = (ILV ? 2 * NT : NT) * 16;
                     const uint32_t b_hi = b_smem + sb * pl.SB;
                     const uint32_t b_lo = ILV ? b_hi + NT * 16 : b_hi + KG * NT * 16;
@@ -241,7 +211,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
                             const uint32_t aoff = (uint32_t)(2 * kk) * RS * 16 + (uint32_t)(mt * 128 + shift) * 16;
                             const uint64_t ah = ptx::smem_desc(a_hi + aoff, RS * 16, 128);
                             const uint64_t al = ptx::smem_desc(a_lo + aoff, RS * 16, 128);
-                            const int accbase = (mt * R + phase) * NACC;
+                            const int accbase = mt * NACC;
                             const uint32_t dh = tmem + (uint32_t)((accbase + chunk % NHH) * NT);
                             const uint32_t dx = tmem + (uint32_t)((accbase + NHH) * NT);
                             const uint32_t acc_h = (chunk >= NHH || !first || kk > 0) ? 1u : 0u;
@@ -298,22 +268,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
         const int pw = ptid >> 5;                  // producer warp 0..15
         const int ch = pw >> 1;                    // channel within the group
         const int lane64 = ((pw & 1) << 5) | lane; // position stride index 0..63
-        const int a_start = (MODE == MODE_CONVT) ? t0 - p.lo : t0 - pad;   // first window row
-        const int xs_start = (MODE == MODE_AMP) ? a_start - 6 : a_start;   // first staged sample
+        const int a_start = t0 - pad;            // first window row
+        const int xs_start = a_start - 6;        // first staged sample
         const int n_start = 2 * a_start - 5;
-        const int XW = (MODE == MODE_AMP) ? ROWS + 12 : ROWS;
+        const int XW = ROWS + 12;
         const int SW = 2 * ROWS + 10;
         const long long xbase = (long long)b * Cin * L;
         const int gtotal = nchunks * KG;
         auto prefetch = [&](int gi) {
-            const long long rowoff = xbase + (long long)(gi * 8 + ch) * L;
-#pragma unroll
-            for (int s = 0; s < NIN; ++s) {
-                if (s > 0 && !mean3) break;
-                const float* src = (s == 0 ? J.x0 : (s == 1 ? J.x1 : J.x2)) + rowoff;
-                float* dst = xs + ((size_t)((gi & 1) * NIN + s) * 8 + ch) * pl.XWs;
-                for (int q = lane64; q < XW; q += 64) ptx::cp_async4(dst + q, src + clampi(xs_start + q, 0, L - 1));
-            }
+            const float* src = J.x0 + xbase + (long long)(gi * 8 + ch) * L;
+            float* dst = xs + ((size_t)(gi & 1) * 8 + ch) * pl.XWs;
+            for (int q = lane64; q < XW; q += 64) ptx::cp_async4(dst + q, src + clampi(xs_start + q, 0, L - 1));
             ptx::cp_async_commit();
         };
         prefetch(0);
@@ -334,8 +299,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
             if (g == 0 && *prod_go == 0) break;
             uint8_t* a_hi = As + (size_t)sa * pl.SA + (size_t)g * RS * 16;
             uint8_t* a_lo = a_hi + (size_t)KG * RS * 16;
-            const float* xg = xs + (size_t)(gi & 1) * NIN * 8 * pl.XWs;
-            if (MODE == MODE_AMP) {
+            const float* xg = xs + (size_t)(gi & 1) * 8 * pl.XWs;
+            {
                 // ---- SnakeBeta of the 2x upsampled signal, one channel per warp pair.  A lane
                 // takes one input position m and forms both phases n = 2m (taps 1,3,..,11 on
                 // x[m+2..m-3]) and n = 2m+1 (taps 0,2,..,10 on x[m+3..m-2]) from the same seven
@@ -410,33 +375,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
                         *reinterpret_cast<uint32_t*>(a_lo + off) = pack_bf16(l[0], l[1]);
                     }
                 }
-            } else {
-                if (gi + 1 < gtotal) prefetch(gi + 1);
-                // ---- plain split of the staged input: one row (8 channels) per thread
-                for (int q = ptid; q < ROWS; q += NPROD) {
-                    const bool in = a_start + q >= 0 && a_start + q < L;   // zero outside the input
-                    float h[8], l[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float v = xg[c * pl.XWs + q];
-                        if (mean3)
-                            v = (v + xg[(8 + c) * pl.XWs + q] + xg[(16 + c) * pl.XWs + q]) / 3.0f;
-                        v = in ? v : 0.f;
-                        h[c] = bf16_round(v);
-                        l[c] = v - h[c];
-                    }
-                    uint4 hv, lv;
-                    hv.x = pack_bf16(h[0], h[1]);
-                    hv.y = pack_bf16(h[2], h[3]);
-                    hv.z = pack_bf16(h[4], h[5]);
-                    hv.w = pack_bf16(h[6], h[7]);
-                    lv.x = pack_bf16(l[0], l[1]);
-                    lv.y = pack_bf16(l[2], l[3]);
-                    lv.z = pack_bf16(l[4], l[5]);
-                    lv.w = pack_bf16(l[6], l[7]);
-                    *reinterpret_cast<uint4*>(a_hi + (size_t)q * 16) = hv;
-                    *reinterpret_cast<uint4*>(a_lo + (size_t)q * 16) = lv;
-                }
             }
             if (g == KG - 1) {
                 ptx::fence_proxy_async_smem();
@@ -460,34 +398,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
         const int q4 = warp & 3;                   // TMEM lane quarter this warp may access
         const int part = (warp - 2) >> 2;          // which quarter of the columns (0..3)
         constexpr int CPP = (NT / 4 >= 16) ? NT / 4 : 16;
-        const int Lout = L * r;
-        const long long obase = (long long)b * Cout * Lout;
+        const long long obase = (long long)b * Cout * L;
         if (epi_go && part * CPP < NT) {
             const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const int row = t0 + mt * 128 + q4 * 32 + lane;
-                for (int phase = 0; phase < R; ++phase) {
-                    const int t = (MODE == MODE_CONVT) ? row * r + phase : row;
-                    for (int cb = part * CPP; cb < part * CPP + CPP && cb < NT; cb += 16) {
-                        float v[16], w[16];
-                        const int accbase = (mt * R + phase) * NACC;
-                        ptx::tmem_ld16(lane_addr + (uint32_t)(accbase * NT + cb), v);
+                const int t = t0 + mt * 128 + q4 * 32 + lane;
+                for (int cb = part * CPP; cb < part * CPP + CPP && cb < NT; cb += 16) {
+                    float v[16], w[16];
+                    const int accbase = mt * NACC;
+                    ptx::tmem_ld16(lane_addr + (uint32_t)(accbase * NT + cb), v);
 #pragma unroll
-                        for (int a = 1; a < NACC; ++a) {
-                            ptx::tmem_ld16(lane_addr + (uint32_t)((accbase + a) * NT + cb), w);
+                    for (int a = 1; a < NACC; ++a) {
+                        ptx::tmem_ld16(lane_addr + (uint32_t)((accbase + a) * NT + cb), w);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) v[i] += w[i];
-                        }
-                        if (row < L) {
+                        for (int i = 0; i < 16; ++i) v[i] += w[i];
+                    }
+                    if (t < L) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int o = o0 + cb + i;
-                                const long long idx = obase + (long long)o * Lout + t;
-                                float y = v[i] + __ldg(J.bias + o);
-                                if (MODE == MODE_AMP && J.res) y += J.res[idx];
-                                J.out[idx] = y;
-                            }
+                        for (int i = 0; i < 16; ++i) {
+                            const int o = o0 + cb + i;
+                            const long long idx = obase + (long long)o * L + t;
+                            float y = v[i] + __ldg(J.bias + o);
+                            if (J.res) y += J.res[idx];
+                            J.out[idx] = y;
                         }
                     }
                 }
@@ -832,7 +766,6 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         const int mt = col0 / NT, oc0 = col0 % NT;
         // regions [mt][phase][NT]: this warp's columns of phase phi start at + phi * NT
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(mt * RSTR + oc0);
-        constexpr bool kPrefetch = (R == 1) && CW <= 16;   // residual loaded ahead of the MMAs
         const long long Lout = (long long)L * R;
         bool ok = *abort_flag == 0;
         int ip = 0;
@@ -850,20 +783,42 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             const int t = T.t0 + mt * 128 + q4 * 32 + lane;   // the row (input sample when R > 1)
             const int o_base = T.ot * NT + oc0;
             const long long idx0 = ((long long)T.b * Cout + o_base) * Lout + (long long)R * t;
-            // this warp's bias values, staged in shared memory while the tile's MMAs run (read
-            // back as broadcasts by the final stores)
+            // The accumulator starts from bias + residual, read at the start of the tile while
+            // its first passes run.  Read after the last pass, they would sit behind the tensor
+            // core's operand traffic for thousands of cycles while the MMA warp waits for this
+            // warp to drain the next tile's passes.  The bias slice goes through shared memory
+            // (CW / 32 loads per lane, then broadcasts).
             float* bsl = bias_s + (warp - 2) * CW;
             for (int c = lane; c < CW; c += 32) bsl[c] = (o_base + c < Cout) ? __ldg(J.bias + o_base + c) : 0.f;
             __syncwarp();
-            float res[kPrefetch ? CW : 1];
-            if (kPrefetch) {
-#pragma unroll
-                for (int c = 0; c < CW; ++c)
-                    res[c] = (J.res && t < L && o_base + c < Cout) ? J.res[idx0 + (long long)c * Lout] : 0.f;
-            }
             float acc[R * CW];
+            {
+                const bool has_res = R == 1 && J.res != nullptr && t < L;
 #pragma unroll
-            for (int c = 0; c < R * CW; ++c) acc[c] = 0.f;
+                for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+                if (has_res && o_base + CW <= Cout) {
+                    const float* rp = J.res + idx0;
+#pragma unroll
+                    for (int c = 0; c < CW; ++c, rp += Lout) acc[c] = __ldg(rp);
+                } else if (NT <= 16 && has_res) {   // only 16-wide tiles pad past Cout
+                    const float* rp = J.res + idx0;
+#pragma unroll
+                    for (int c = 0; c < CW; ++c, rp += Lout)
+                        if (o_base + c < Cout) acc[c] = __ldg(rp);
+                }
+#pragma unroll
+                for (int cb = 0; cb < CW; cb += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(bsl + cb);
+                    acc[cb] += b4.x;
+                    acc[cb + 1] += b4.y;
+                    acc[cb + 2] += b4.z;
+                    acc[cb + 3] += b4.w;
+                }
+#pragma unroll
+                for (int ph = 1; ph < R; ++ph)
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) acc[ph * CW + c] = acc[c];
+            }
             for (int ps = 0; ps < npass; ++ps, ++ip) {
                 const int buf = ip & 1;
                 if (!ptx::mbar_wait(&acc_full[buf], (ip >> 1) & 1, kWaitLimit)) { ok = false; break; }
@@ -893,27 +848,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                 break;
             }
             if (t < L) {
-                // FC channels at a time: all residual loads of a group are in flight before its
-                // stores
-                constexpr int FC = (R * CW > 64) ? 8 : 16;
-                const bool has_res = R == 1 && J.res != nullptr;
 #pragma unroll
-                for (int cb = 0; cb < CW; cb += FC) {
-                    float rs[FC];
+                for (int c = 0; c < CW; ++c) {
+                    if (NT <= 16 && o_base + c >= Cout) continue;   // channels past Cout pad the tile
 #pragma unroll
-                    for (int c = 0; c < FC; ++c) {
-                        const int o = o_base + cb + c;   // channels past Cout pad the tile
-                        if (kPrefetch) rs[c] = res[cb + c];
-                        else rs[c] = (has_res && o < Cout) ? J.res[idx0 + (long long)(cb + c) * Lout] : 0.f;
-                    }
-#pragma unroll
-                    for (int c = 0; c < FC; ++c) {
-                        if (o_base + cb + c >= Cout) continue;
-                        const float bb = bsl[cb + c];
-#pragma unroll
-                        for (int ph = 0; ph < R; ++ph)
-                            J.out[idx0 + (long long)(cb + c) * Lout + ph] = (acc[ph * CW + cb + c] + bb) + rs[c];
-                    }
+                    for (int ph = 0; ph < R; ++ph) J.out[idx0 + (long long)c * Lout + ph] = acc[ph * CW + c];
                 }
             }
             __syncwarp();   // the bias slice is rewritten for the next tile
@@ -958,49 +897,33 @@ int ntile_convt(int Cout, int r) {
 // 8-channel groups per K chunk of an upsampler: 32-channel chunks, or one 16-channel chunk.
 int kgt_convt(int Cin) { return Cin % 32 == 0 ? 4 : (Cin == 16 ? 2 : 0); }
 
-template <int MODE, int MT, int NT, int NIN>
+template <int MT, int NT>
 TcPlan make_plan(const TcParams& p, int njobs) {
     int span = 0;
-    if (MODE == MODE_CONVT) {
-        // tap shifts (phi + pad - j) / r + lo span [0, span]
-        const int K = p.job[0].K, pad = p.job[0].pad, r = p.r;
-        int smax = -1000000, smin = 1000000;
-        for (int j = 0; j < K; ++j) {
-            const int phase = ((j - pad) % r + r) % r;
-            const int a = phase + pad - j;
-            const int s = a >= 0 ? a / r : -((-a + r - 1) / r);
-            smax = std::max(smax, s);
-            smin = std::min(smin, s);
-        }
-        span = smax - smin;
-    } else {
-        for (int j = 0; j < njobs; ++j) span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
-    }
+    for (int j = 0; j < njobs; ++j) span = std::max(span, (p.job[j].K - 1) * p.job[j].dil);
     TcPlan pl{};
     pl.RS = 128 * MT + span;
     pl.XWs = pl.RS + 12;
-    pl.SWs = (MODE == MODE_AMP) ? 2 * pl.RS + 12 : 0;   // even (8-byte rows), room for the last pair
+    pl.SWs = 2 * pl.RS + 12;   // even (8-byte rows), room for the last pair
     pl.SA = 2 * KG * pl.RS * 16;
     pl.SB = 2 * KG * NT * 16;
     pl.offB = NSA * pl.SA;
     pl.offX = pl.offB + NSB * pl.SB;
-    const int stage_bytes = (2 * NIN * 8 * pl.XWs + 8 * pl.SWs) * 4;
+    const int stage_bytes = (2 * 8 * pl.XWs + 8 * pl.SWs) * 4;
     pl.offBar = (pl.offX + stage_bytes + 15) / 16 * 16;
     pl.smem = pl.offBar + 8 * (2 * NSA + 2 * NSB + 1) + 16;
     return pl;
 }
 
-template <int MODE, int MT, int NT, int NACC, int R>
+template <int MT, int NT, int NACC>
 int launch_tc(const TcParams& p0, int njobs, cudaStream_t s) {
     TcParams p = p0;
     if (NACC - 1 > p.Cin / KC) return -1;  // every head accumulator must receive a chunk
     if (p.Cin % KC != 0 || p.Cout % NT != 0) return -1;
-    if (MODE == MODE_CONVT && p.r != R) return -1;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
-    constexpr int NIN = (MODE == MODE_CONVT) ? 3 : 1;
-    const TcPlan pl = make_plan<MODE, MT, NT, NIN>(p, njobs);
+    const TcPlan pl = make_plan<MT, NT>(p, njobs);
     if (pl.smem > 227 * 1024) return -1;
-    auto kern = k_conv_tc<MODE, MT, NT, NACC, R>;
+    auto kern = k_conv_tc<MT, NT, NACC>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess) return -1;
     dim3 grid(p.tiles_t * p.B, p.Cout / NT, njobs);
     kern<<<grid, NTHREADS, pl.smem, s>>>(p, pl);
@@ -1013,11 +936,11 @@ int launch_tc(const TcParams& p0, int njobs, cudaStream_t s) {
 // and a single head accumulator (stage-0 relative error about 4e-5, against 1e-5 with three).
 int dispatch_amp(const TcParams& p, int njobs, cudaStream_t s) {
     switch (p.Cin) {
-        case 512: return launch_tc<MODE_AMP, 1, 256, 2, 1>(p, njobs, s);
-        case 256: return launch_tc<MODE_AMP, 1, 256, 2, 1>(p, njobs, s);
-        case 128: return launch_tc<MODE_AMP, 1, 128, 4, 1>(p, njobs, s);
-        case 64: return launch_tc<MODE_AMP, 2, 64, 3, 1>(p, njobs, s);
-        case 32: return launch_tc<MODE_AMP, 2, 32, 2, 1>(p, njobs, s);
+        case 512: return launch_tc<1, 256, 2>(p, njobs, s);
+        case 256: return launch_tc<1, 256, 2>(p, njobs, s);
+        case 128: return launch_tc<1, 128, 4>(p, njobs, s);
+        case 64: return launch_tc<2, 64, 3>(p, njobs, s);
+        case 32: return launch_tc<2, 32, 2>(p, njobs, s);
         default: return -1;
     }
 }
@@ -1041,6 +964,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     GemmParams p = p0;
     const int kc = 8 * KGT;
     if (p.Cin % kc != 0 || njobs < 1 || !p.sched || !p.err) return -1;
+    if (NT > 16 && p.Cout % NT != 0) return -1;   // the epilogue pads channels past Cout only in 16-wide tiles
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
     int span = 0, kumax = 1;
     for (int j = 0; j < njobs; ++j) {
@@ -1159,8 +1083,6 @@ void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, bool interleave
 TcJob make_job(const ConvJob& J, const TcConv& tw) {
     TcJob T{};
     T.x0 = J.x0;
-    T.x1 = J.x1;
-    T.x2 = J.x2;
     T.w = reinterpret_cast<const uint16_t*>(tw.dev);
     T.bias = J.bias;
     T.alpha = J.alpha;
@@ -1233,7 +1155,6 @@ int launch_conv_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int
     p.Cout = cp.Cout;
     p.L = cp.L;
     p.B = cp.B;
-    p.r = 1;
     p.filt = cp.filt;
     p.err = err;
     // heaviest kernel first (blockIdx.z = 0), so the longest blocks start earliest
