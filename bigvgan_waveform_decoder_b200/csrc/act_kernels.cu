@@ -56,9 +56,17 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
     float* xs = buf + c * XF_P;
     float* T = buf + 8 * XF_P;   // [8][TF_P] outputs, skewed
     const float* xrow = J.x + ((long long)b * p.C + g * 8 + c) * L;
-    // all of the window's loads in flight at once (asynchronous copies straight to shared);
-    // skew(lane + 32 k) = skew(lane) + 40 k
-    {
+    // all of the window's loads in flight at once (asynchronous copies straight to shared)
+    if (!EDGE && (reinterpret_cast<uintptr_t>(xrow + t0 - 8) & 15) == 0) {
+        // 16-byte copies (the window starts on a 16-byte boundary; a skewed group of 4 floats
+        // stays contiguous and 16-byte aligned in shared memory)
+#pragma unroll
+        for (int k = 0; k < (XF / 4 + 31) / 32; ++k) {
+            const int i = 4 * (lane + 32 * k);
+            if (i < XF) ptx::cp_async16(xs + skew(i), xrow + t0 - 8 + i);
+        }
+    } else {
+        // skew(lane + 32 k) = skew(lane) + 40 k
         float* dst = xs + skew(lane);
 #pragma unroll
         for (int k = 0; k < (XF + 31) / 32; ++k) {
@@ -132,8 +140,8 @@ __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
     }
 }
 
-// Plain head/tail split (no activation) into the same row layout, of x0 or of the mean
-// (x0 + x1 + x2) / 3 of three block outputs.  grid: x = row tiles of NT_ACT, y = B * C / 8.
+// Plain head/tail split (no activation) into the same row layout, of x0, of the mean
+// (x0 + x1 + x2) / 3 of three block outputs, or of the sum of four partial outputs.  grid: x = row tiles of NT_ACT, y = B * C / 8.
 __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
     const int L = p.L, ngroups = p.C / 8;
     const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
@@ -147,7 +155,9 @@ __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const long long i = base + (long long)c * L;
-            v[c] = p.x1 ? (__ldg(p.x0 + i) + __ldg(p.x1 + i) + __ldg(p.x2 + i)) / 3.0f : __ldg(p.x0 + i);
+            if (p.x3) v[c] = ((__ldg(p.x0 + i) + __ldg(p.x1 + i)) + __ldg(p.x2 + i)) + __ldg(p.x3 + i);
+            else if (p.x1) v[c] = (__ldg(p.x0 + i) + __ldg(p.x1 + i) + __ldg(p.x2 + i)) / 3.0f;
+            else v[c] = __ldg(p.x0 + i);
         }
     } else {
 #pragma unroll
@@ -166,7 +176,7 @@ __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
 
 int launch_split_rows(const SplitParams& p, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0 || !p.x0) return -1;
-    if ((p.x1 == nullptr) != (p.x2 == nullptr)) return -1;
+    if ((p.x1 == nullptr) != (p.x2 == nullptr) || (p.x3 && !p.x1)) return -1;
     const int total = p.L + p.pad_l + p.pad_r;
     dim3 grid((total + NT_ACT - 1) / NT_ACT, p.B * (p.C / 8));
     k_split_rows<<<grid, NT_ACT, 0, s>>>(p);

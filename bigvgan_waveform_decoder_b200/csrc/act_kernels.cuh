@@ -24,6 +24,7 @@ struct SplitParams {
     const float* x0;        // [B, C, L] fp32
     const float* x1;        // with x2: split the mean (x0 + x1 + x2) / 3 instead (else null)
     const float* x2;
+    const float* x3;        // with x1, x2: split the sum ((x0 + x1) + x2) + x3 instead (else null)
     void* a_hi;             // [B, C/8, pad_l + L + pad_r] rows of 8 bf16 (heads)
     void* a_lo;             // same shape (tails)
     int C, L, B;
@@ -36,5 +37,6 @@ int launch_split_rows(const SplitParams& p, cudaStream_t s);
 // One launch for `njobs` activations of the same shape (blockIdx.z = job).  Returns the number
 // of kernels launched or -1.
 int launch_act_split(const ActParams& p, int njobs, cudaStream_t s);
+
 
 }  // namespace mh3a

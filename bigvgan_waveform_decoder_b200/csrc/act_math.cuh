@@ -1,5 +1,6 @@
-// act_math.cuh -- the anti-aliased SnakeBeta of one channel, register-blocked per lane, shared by
-// the standalone activation kernel and the producer warps of the fused tensor-core GEMM.
+// act_math.cuh -- the anti-aliased SnakeBeta of one channel, register-blocked per lane (the
+// standalone activation kernel), and the sine of SnakeBeta that the producer warps of the fused
+// tensor-core AMP kernel share with it.
 //
 //   a = down2(snake(up2(x)))      (FastVideo "minimax_h3_audio_vae" page, `_activation1d`;
 //                                  filter from `kaiser_sinc_filter1d`)

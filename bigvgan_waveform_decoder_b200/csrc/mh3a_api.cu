@@ -122,6 +122,7 @@ struct mh3a_handle {
     long long stage_cap = 0;   // floats per stage buffer
     float* buf_in = nullptr;   // [B, latent_dim, N]
     float* buf_pre = nullptr;  // [B, decoder_dim, N]
+    float* pre_part[4] = {};   // conv_pre's partial outputs on the tensor-core path
     float* H = nullptr;
     float* X[MH3A_MAX_RESBLOCKS] = {};
     float* T[MH3A_MAX_RESBLOCKS] = {};
@@ -364,9 +365,21 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
     return MH3A_OK;
 }
 
-// Head/tail rows of x0 (or of the mean of x0, x1, x2) into the first A operand pair.
+// The kPreSplit partial outputs of the tensor-core conv_pre: buf_pre (with the bias), then three
+// stage buffers that are free until the first AMP stage (sized for decoder_dim x N at create).
+float* const* pre_parts(mh3a_handle* h) {
+    static_assert(kPreSplit == 4, "four partial buffers");
+    h->pre_part[0] = h->buf_pre;
+    h->pre_part[1] = h->H;
+    h->pre_part[2] = h->X[0];
+    h->pre_part[3] = h->T[0];
+    return h->pre_part;
+}
+
+// Head/tail rows of x0 (or of the mean of x0, x1, x2, or of the sum of x0 .. x3) into the first
+// A operand pair.
 mh3a_status split_to_a(mh3a_handle* h, const float* x0, const float* x1, const float* x2, int C, int L, int B,
-                       cudaStream_t s) {
+                       cudaStream_t s, const float* x3 = nullptr) {
     if ((long long)B * C * ((long long)L + kApadL + kApadR) > h->a_cap) {
         g_last_error = "batch too large for the tensor-core operand buffers (B > max_batch)";
         return MH3A_ERR_SHAPE;
@@ -375,6 +388,7 @@ mh3a_status split_to_a(mh3a_handle* h, const float* x0, const float* x1, const f
     sp.x0 = x0;
     sp.x1 = x1;
     sp.x2 = x2;
+    sp.x3 = x3;
     sp.a_hi = h->A_hi[0];
     sp.a_lo = h->A_lo[0];
     sp.C = C;
@@ -426,7 +440,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             // split the input into head/tail rows once, then the persistent tensor-core GEMM
             if ((st = split_to_a(h, h->buf_in, nullptr, nullptr, c.latent_dim, N, B, s))) return st;
             n = launch_conv_pre_gemm(p, h->tc[0], h->A_hi[0], h->A_lo[0], kApadL, (long long)N + kApadL + kApadR,
-                                     s, h->dev_err, h->dev_err + 16);
+                                     pre_parts(h), s, h->dev_err, h->dev_err + 16);
         } else {
             n = launch_conv_simt(p, 1, false, false, s);
         }
@@ -455,7 +469,14 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             return MH3A_ERR_UNSUPPORTED;
         }
         int nl;
-        if (h->ups_tc[i]) {
+        if (i == 0 && h->pre_tc) {
+            // conv_pre left its output as partial sums over input-channel slices
+            float* const* part = pre_parts(h);
+            if (!h->ups_tc[i]) return MH3A_ERR_UNSUPPORTED;
+            if ((st = split_to_a(h, part[0], part[1], part[2], C, L, B, s, part[3]))) return st;
+            nl = launch_convT_gemm(q, h->tc[i], h->A_hi[0], h->A_lo[0], kApadL, (long long)L + kApadL + kApadR, s,
+                                   h->dev_err, h->dev_err + 16);
+        } else if (h->ups_tc[i]) {
             if ((st = split_to_a(h, q.x0, q.x1, q.x2, C, L, B, s))) return st;
             nl = launch_convT_gemm(q, h->tc[i], h->A_hi[0], h->A_lo[0], kApadL, (long long)L + kApadL + kApadR, s,
                                    h->dev_err, h->dev_err + 16);
@@ -675,7 +696,10 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
         if (!v) return fail(MH3A_ERR_MISSING_WEIGHT);
         if (v->ndim != 3 || v->shape[2] != 7) return fail(MH3A_ERR_SHAPE);
         std::vector<float> oik;
-        h->pre_tc = c.precision == MH3A_BF16X3 && tc_pre_supported(c.decoder_dim, c.latent_dim, 7);
+        // the tensor-core conv_pre leaves partial sums that only the tensor-core upsampler's
+        // input split reduces
+        h->pre_tc = c.precision == MH3A_BF16X3 && tc_pre_supported(c.decoder_dim, c.latent_dim, 7) &&
+                    c.n_stages >= 1 && tc_convt_supported(c.decoder_dim, c.decoder_dim / 2, c.rates[0], c.kernels[0]);
         if ((st = fold_conv(lk, "decoder.conv_pre", c.decoder_dim, c.latent_dim, 7, true, ha, &h->pre,
                             h->pre_tc ? &oik : nullptr)))
             return fail(st);
@@ -744,6 +768,8 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     }
     const long long BN = (long long)c.max_batch * c.max_frames;
     h->stage_cap = ((cap * BN + 63) / 64) * 64;
+    if (h->pre_tc)   // three stage buffers also hold conv_pre's partial outputs
+        h->stage_cap = std::max(h->stage_cap, (((long long)c.decoder_dim * BN + 63) / 64) * 64);
     auto rnd = [](long long n) { return ((n + 63) / 64) * 64; };
     const long long n_in = rnd((long long)c.latent_dim * BN), n_pre = rnd((long long)c.decoder_dim * BN);
     const long long n_lat = rnd((long long)c.latent_channels * BN), n_wav = rnd((long long)h->hop * BN);

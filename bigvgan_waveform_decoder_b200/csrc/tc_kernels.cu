@@ -35,6 +35,7 @@
 #include <algorithm>
 #include <cstring>
 
+#include "act_math.cuh"
 #include "tc_kernels.cuh"
 #include "tc_ptx.cuh"
 
@@ -86,20 +87,6 @@ __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? l
 // narrow tile is bound by reading that operand from shared memory).  Their weight blocks store
 // each core column's head rows directly followed by its tail rows.
 __host__ __device__ constexpr bool interleaved_b(int NT, int R) { return R == 1 && NT <= 64; }
-
-// sin^2(alpha u) for the tensor-core path: Cody-Waite reduction modulo pi, then the hardware
-// sine on [-pi/2, pi/2] (absolute error near 2^-21, far below the 3xBF16 operand error).
-__device__ __forceinline__ float sin_sq_fast(float alpha, float u) {
-    const float kInvPi = 0.318309886183790671538f;
-    const float kPiHi = 3.14159274101257324219f;
-    const float kPiLo = -8.74227800037248297e-08f;
-    const float v = alpha * u;
-    const float k = rintf(v * kInvPi);
-    float r = fmaf(-k, kPiHi, v);
-    r = fmaf(-k, kPiLo, r);
-    const float s = __sinf(r);
-    return s * s;
-}
 
 __device__ __forceinline__ void prod_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NPROD) : "memory"); }
 
@@ -322,8 +309,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_conv_tc(const TcParams p, const
                             ue = fmaf(p.filt.up[2 * k + 1], xv[5 - k], ue);
                             uo = fmaf(p.filt.up[2 * k], xv[6 - k], uo);
                         }
-                        const float se = fmaf(sin_sq_fast(al, ue), ib, ue);
-                        const float so = fmaf(sin_sq_fast(al, uo), ib, uo);
+                        const float se = fmaf(actm::sin_sq_fast(al, ue), ib, ue);
+                        const float so = fmaf(actm::sin_sq_fast(al, uo), ib, uo);
                         const int ie = 2 * m - n_start;
                         const float ve = (m > L - 1) ? so : se;
                         const float vo = (m < 0) ? se : so;
@@ -449,6 +436,7 @@ struct GemmJob {
     const float* res;
     float* out;
     int K, dil, pad;
+    int g0;               // first 8-channel group of the job's input-channel slice
     int span;             // window rows a tile reads beyond its 128 MT output rows
     // polyphase transposed conv (R > 1): window row offset and output phase of every tap
     int8_t tap_row[16];
@@ -458,6 +446,7 @@ struct GemmJob {
 struct GemmParams {
     GemmJob job[MH3A_MAX_RESBLOCKS];
     int Cin, Cout, L, B, tiles_t;
+    int a_groups;         // 8-channel groups per item in the A arrays (Cin / 8 unless split)
     int pad_l;            // zero rows before the sequence in the A arrays
     long long Lpad;       // rows per (item, channel group) in the A arrays
     int tpu;              // tap units per weight bulk copy (set by the launcher)
@@ -513,6 +502,33 @@ __device__ __forceinline__ PsTile ps_tile(const GemmParams& p, const PsSched& sc
     return T;
 }
 
+
+// Residual group g (channels GW g .. GW g + GW - 1 of a warp's columns) of one row, rp = the row's
+// first column; channels past Cout (16-wide tiles only) read nothing.
+template <int NT, int GW>
+__device__ __forceinline__ void load_res_group(float (&rq)[GW], const float* rp, int g, long long Lout, int o_base,
+                                               int Cout) {
+#pragma unroll
+    for (int c = 0; c < GW; ++c) {
+        const int cc = GW * g + c;
+        rq[c] = (NT > 16 || o_base + cc < Cout) ? __ldg(rp + (long long)cc * Lout) : 0.f;
+    }
+}
+
+// acc[GW g + c] += rq[c] with a run-time g: one compile-time branch per group keeps every
+// accumulator index a constant (and the accumulators in registers).  The adds are volatile asm
+// so that they stay ahead of the tensor-memory loads that follow them, which would otherwise
+// need registers while rq is still live.
+template <int CW, int GW, int N>
+__device__ __forceinline__ void add_res_group(float (&acc)[N], const float (&rq)[GW], int g) {
+#pragma unroll
+    for (int gg = 0; gg < CW / GW; ++gg) {
+        if (gg == g) {
+#pragma unroll
+            for (int c = 0; c < GW; ++c) asm volatile("add.rn.f32 %0, %0, %1;" : "+f"(acc[GW * gg + c]) : "f"(rq[c]));
+        }
+    }
+}
 
 // KGT = 8-channel groups per K chunk (4: 32 input channels; 2: 16).  KGT = 1 serves 8-channel
 // layers: one MMA K-step of 16 then covers the same 8 channels at two consecutive taps -- the
@@ -722,7 +738,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     for (int part = 0; part < 2; ++part) {
                         const uint8_t* base = part == 0 ? J.a_hi : J.a_lo;
                         for (int g = 0; g < KGT; ++g) {
-                            const long long grp = (long long)T.b * (Cin / 8) + chunk * KGT + g;
+                            const long long grp = (long long)T.b * p.a_groups + J.g0 + chunk * KGT + g;
                             ptx::bulk_g2s(As + (size_t)sa * pl.SA + ((size_t)(part * KGT + g) * RS) * 16,
                                           base + (grp * p.Lpad + row0) * 16, (uint32_t)(ROWS * 16), &a_full[sa]);
                         }
@@ -783,65 +799,96 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             const int t = T.t0 + mt * 128 + q4 * 32 + lane;   // the row (input sample when R > 1)
             const int o_base = T.ot * NT + oc0;
             const long long idx0 = ((long long)T.b * Cout + o_base) * Lout + (long long)R * t;
-            // The accumulator starts from bias + residual, read at the start of the tile while
-            // its first passes run.  Read after the last pass, they would sit behind the tensor
-            // core's operand traffic for thousands of cycles while the MMA warp waits for this
-            // warp to drain the next tile's passes.  The bias slice goes through shared memory
-            // (CW / 32 loads per lane, then broadcasts).
+            // The accumulator starts from bias + residual.  Wide warps (CW >= 64) stream the
+            // residual in, 16 channels per pass, each group loaded after one pass's drain and
+            // added at the next: read at the tile's start, those reads would queue behind the
+            // tensor core's operand traffic while the MMA warp waits for the first drain.
+            // Narrow warps read their few residual values at the tile's start.  The bias slice
+            // goes through shared memory (CW / 32 loads per lane, then broadcasts).
+            constexpr bool kSpread = R == 1 && CW >= 64;
+            constexpr int GW = 16;                            // residual group width
+            constexpr int G = CW / GW;                        // residual groups per warp
+            const bool has_res = R == 1 && J.res != nullptr && t < L;
+            const float* rp = has_res ? J.res + idx0 : nullptr;
             float* bsl = bias_s + (warp - 2) * CW;
-            for (int c = lane; c < CW; c += 32) bsl[c] = (o_base + c < Cout) ? __ldg(J.bias + o_base + c) : 0.f;
+            for (int c = lane; c < CW; c += 32) bsl[c] = (J.bias && o_base + c < Cout) ? __ldg(J.bias + o_base + c) : 0.f;
             __syncwarp();
             float acc[R * CW];
-            {
-                const bool has_res = R == 1 && J.res != nullptr && t < L;
 #pragma unroll
-                for (int c = 0; c < CW; ++c) acc[c] = 0.f;
-                if (has_res && o_base + CW <= Cout) {
-                    const float* rp = J.res + idx0;
+            for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+            if (!kSpread && has_res) {
+                if (NT > 16 || o_base + CW <= Cout) {
 #pragma unroll
-                    for (int c = 0; c < CW; ++c, rp += Lout) acc[c] = __ldg(rp);
-                } else if (NT <= 16 && has_res) {   // only 16-wide tiles pad past Cout
-                    const float* rp = J.res + idx0;
+                    for (int c = 0; c < CW; ++c) acc[c] = __ldg(rp + (long long)c * Lout);
+                } else {   // only 16-wide tiles pad past Cout
 #pragma unroll
-                    for (int c = 0; c < CW; ++c, rp += Lout)
-                        if (o_base + c < Cout) acc[c] = __ldg(rp);
+                    for (int c = 0; c < CW; ++c)
+                        if (o_base + c < Cout) acc[c] = __ldg(rp + (long long)c * Lout);
                 }
-#pragma unroll
-                for (int cb = 0; cb < CW; cb += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(bsl + cb);
-                    acc[cb] += b4.x;
-                    acc[cb + 1] += b4.y;
-                    acc[cb + 2] += b4.z;
-                    acc[cb + 3] += b4.w;
-                }
-#pragma unroll
-                for (int ph = 1; ph < R; ++ph)
-#pragma unroll
-                    for (int c = 0; c < CW; ++c) acc[ph * CW + c] = acc[c];
             }
+#pragma unroll
+            for (int cb = 0; cb < CW; cb += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(bsl + cb);
+                acc[cb] += b4.x;
+                acc[cb + 1] += b4.y;
+                acc[cb + 2] += b4.z;
+                acc[cb + 3] += b4.w;
+            }
+#pragma unroll
+            for (int ph = 1; ph < R; ++ph)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) acc[ph * CW + c] = acc[c];
+            float rq[kSpread ? GW : 1];
             for (int ps = 0; ps < npass; ++ps, ++ip) {
                 const int buf = ip & 1;
                 if (!ptx::mbar_wait(&acc_full[buf], (ip >> 1) & 1, kWaitLimit)) { ok = false; break; }
                 ptx::tc_fence_after();
+                // the group loaded after the previous pass (added before the drain, so that its
+                // registers are free again during the drain)
+                if constexpr (kSpread)
+                    if (has_res && ps >= 1 && ps <= G) add_res_group<CW, GW>(acc, rq, ps - 1);
 #pragma unroll
                 for (int ph = 0; ph < R; ++ph) {
+                    if constexpr (kSpread) {
+                        // 8 columns at a time: the residual group holds 16 registers here
 #pragma unroll
-                    for (int cb = 0; cb < CW; cb += 16) {
-                        float v[16];
-                        ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
-                        if (ILV) {
-                            float x[16];
-                            ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + NT + cb), x);
+                        for (int cb = 0; cb < CW; cb += 8) {
+                            float v[8];
+                            ptx::tmem_ld8(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
 #pragma unroll
-                            for (int c = 0; c < 16; ++c) v[c] += x[c];
+                            for (int c = 0; c < 8; ++c) acc[ph * CW + cb + c] += v[c];
                         }
+                    } else {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) acc[ph * CW + cb + c] += v[c];
+                        for (int cb = 0; cb < CW; cb += 16) {
+                            float v[16];
+                            ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
+                            if (ILV) {
+                                float x[16];
+                                ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + NT + cb), x);
+#pragma unroll
+                                for (int c = 0; c < 16; ++c) v[c] += x[c];
+                            }
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) acc[ph * CW + cb + c] += v[c];
+                        }
                     }
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+                if constexpr (kSpread)
+                    if (has_res && ps < G) load_res_group<NT, GW>(rq, rp, ps, Lout, o_base, Cout);
+            }
+            if constexpr (kSpread) {
+                if (has_res && ok && npass <= G) {
+                    // fewer passes than groups: the last loaded group and the ones never loaded
+                    if (npass >= 1) add_res_group<CW, GW>(acc, rq, npass - 1);
+                    for (int g = npass; g < G; ++g) {
+                        load_res_group<NT, GW>(rq, rp, g, Lout, o_base, Cout);
+                        add_res_group<CW, GW>(acc, rq, g);
+                    }
+                }
             }
             if (!ok || *abort_flag) {
                 ok = false;
@@ -888,7 +935,7 @@ float bf16_value(uint16_t h) {
 
 // Output-channel tile of each layer kind (the weight blocks are laid out for it).
 int ntile_amp(int C) { return C >= 256 ? 256 : (C >= 128 ? 128 : (C >= 64 ? 64 : C)); }
-int ntile_pre(int) { return 64; }
+int ntile_pre(int) { return 256; }
 int ntile_convt(int Cout, int r) {
     if (r > 2) return Cout >= 32 ? 32 : Cout;
     return Cout >= 64 ? 64 : (Cout > 16 ? Cout : 16);   // narrow outputs padded to 16 columns
@@ -965,6 +1012,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     const int kc = 8 * KGT;
     if (p.Cin % kc != 0 || njobs < 1 || !p.sched || !p.err) return -1;
     if (NT > 16 && p.Cout % NT != 0) return -1;   // the epilogue pads channels past Cout only in 16-wide tiles
+    if (p.a_groups == 0) p.a_groups = p.Cin / 8;
     p.tiles_t = (p.L + 128 * MT - 1) / (128 * MT);
     int span = 0, kumax = 1;
     for (int j = 0; j < njobs; ++j) {
@@ -1108,7 +1156,9 @@ bool tc_stage_supported(int C, const mh3a_config& c) {
     return true;
 }
 
-bool tc_pre_supported(int Cout, int Cin, int k) { return Cout % 64 == 0 && Cin % KC == 0 && Cin >= 7 * KC && k <= 15; }
+bool tc_pre_supported(int Cout, int Cin, int k) {
+    return Cout % 256 == 0 && Cin % (32 * kPreSplit) == 0 && k <= 15;
+}
 
 bool tc_convt_supported(int Cin, int Cout, int r, int K) {
     const int kgt = kgt_convt(Cin);
@@ -1130,9 +1180,10 @@ void prepare_tc_conv(const std::vector<float>& w, int C, int k, TcConv* out) {
 }
 
 void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWeights* out) {
-    pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + c) * k + tap]; }, O, I, k, ntile_pre(O), KG,
-                interleaved_b(ntile_pre(O), 1),
-                &out->pre);
+    const int Is = I / kPreSplit;   // input channels per slice
+    for (int sl = 0; sl < kPreSplit; ++sl)
+        pack_blocks([&](int o, int c, int tap) { return w[((size_t)o * I + sl * Is + c) * k + tap]; }, O, Is, k,
+                    ntile_pre(O), 4, interleaved_b(ntile_pre(O), 1), &out->pre[sl]);
 }
 
 void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
@@ -1144,7 +1195,7 @@ void tc_finalize(TcStageWeights* w) {
     for (auto& a : w->conv)
         for (auto& b : a)
             for (auto& c : b) std::vector<float>().swap(c.staging);
-    std::vector<float>().swap(w->pre.staging);
+    for (auto& c : w->pre) std::vector<float>().swap(c.staging);
     std::vector<float>().swap(w->ups.staging);
 }
 
@@ -1209,29 +1260,34 @@ int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w,
 
 
 int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                         int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched) {
-    if (!w.pre.dev || cp.Cout % ntile_pre(cp.Cout) != 0) return -1;
+                         int pad_l, long long Lpad, float* const* part, cudaStream_t s, int* err, int* sched) {
+    if (cp.Cout % ntile_pre(cp.Cout) != 0 || cp.Cin % (32 * kPreSplit) != 0) return -1;
     GemmParams p{};
     p.sched = sched;
-    p.Cin = cp.Cin;
+    p.Cin = cp.Cin / kPreSplit;       // the K range of one job
+    p.a_groups = cp.Cin / 8;
     p.Cout = cp.Cout;
     p.L = cp.L;
     p.B = cp.B;
     p.pad_l = pad_l;
     p.Lpad = Lpad;
     p.err = err;
-    GemmJob& G = p.job[0];
-    G.a_hi = static_cast<const uint8_t*>(a_hi);
-    G.a_lo = static_cast<const uint8_t*>(a_lo);
-    G.w = reinterpret_cast<const uint16_t*>(w.pre.dev);
-    G.bias = cp.job[0].bias;
-    G.res = nullptr;
-    G.out = cp.job[0].out;
-    G.K = cp.job[0].K;
-    G.dil = cp.job[0].dil;
-    G.pad = cp.job[0].pad;
-    G.span = (G.K - 1) * G.dil;
-    return launch_gemm_ps<1, 64, 4, 16, 1>(p, 1, s);
+    for (int sl = 0; sl < kPreSplit; ++sl) {
+        if (!w.pre[sl].dev || !part[sl]) return -1;
+        GemmJob& G = p.job[sl];
+        G.a_hi = static_cast<const uint8_t*>(a_hi);
+        G.a_lo = static_cast<const uint8_t*>(a_lo);
+        G.w = reinterpret_cast<const uint16_t*>(w.pre[sl].dev);
+        G.bias = sl == 0 ? cp.job[0].bias : nullptr;
+        G.res = nullptr;
+        G.out = part[sl];
+        G.K = cp.job[0].K;
+        G.dil = cp.job[0].dil;
+        G.pad = cp.job[0].pad;
+        G.g0 = sl * (p.Cin / 8);
+        G.span = (G.K - 1) * G.dil;
+    }
+    return launch_gemm_ps<1, 256, 4, 8, 1>(p, kPreSplit, s);
 }
 
 int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,

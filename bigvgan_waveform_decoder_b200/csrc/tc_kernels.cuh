@@ -15,10 +15,15 @@ struct TcConv {
     int cout = 0, cin = 0, k = 0;
 };
 
+// conv_pre is split along its input channels into kPreSplit slices (jobs of one launch, each
+// writing a partial output that the next layer's input split sums).
+constexpr int kPreSplit = 4;
+static_assert(kPreSplit <= MH3A_MAX_RESBLOCKS, "one GEMM job per slice");
+
 struct TcStageWeights {
     TcConv conv[MH3A_MAX_RESBLOCKS][MH3A_MAX_DILATIONS][2];  // AMP convs of the stage
     TcConv ups;                                             // the stage's transposed conv
-    TcConv pre;                                             // conv_pre (stage 0 only)
+    TcConv pre[kPreSplit];                                  // conv_pre slices (stage 0 only)
 };
 
 // Which layers run on the tensor cores.
@@ -39,7 +44,8 @@ void tc_register(TcStageWeights* w, AddFn add) {
             for (auto& c : b)
                 if (!c.staging.empty()) add(c.staging, &c.dev);
     if (!w->ups.staging.empty()) add(w->ups.staging, &w->ups.dev);
-    if (!w->pre.staging.empty()) add(w->pre.staging, &w->pre.dev);
+    for (auto& c : w->pre)
+        if (!c.staging.empty()) add(c.staging, &c.dev);
 }
 
 // Drop host staging once the device copy exists.
@@ -61,8 +67,10 @@ int launch_amp_gemm_tc(const ConvParams& p, int njobs, const TcStageWeights& w, 
 
 // conv_pre and the upsamplers on the persistent GEMM, reading their input as pre-split rows
 // (launch_split_rows) with pad_l zero rows before the sequence and Lpad rows per channel group.
+// conv_pre writes kPreSplit partial outputs: part[0] = cp.job[0].out (with the bias), part[s]
+// for s >= 1 (input-channel slice s, no bias); their sum is the conv's output.
 int launch_conv_pre_gemm(const ConvParams& cp, const TcStageWeights& w, const void* a_hi, const void* a_lo,
-                         int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched);
+                         int pad_l, long long Lpad, float* const* part, cudaStream_t s, int* err, int* sched);
 int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void* a_hi, const void* a_lo,
                       int pad_l, long long Lpad, cudaStream_t s, int* err, int* sched);
 
