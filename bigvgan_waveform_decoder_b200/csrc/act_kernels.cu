@@ -172,7 +172,150 @@ __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
     reinterpret_cast<uint4*>(p.a_lo)[row] = lv;
 }
 
+// grid: x = row tiles of NT_ACT, y = B * C / 8.  The group's 8 x Cz weights and 8 biases sit in
+// shared memory (read back as broadcasts); every thread forms one row of 8 channels.
+__global__ void __launch_bounds__(NT_ACT) k_proj_split(const ProjSplitParams p) {
+    __shared__ __align__(16) float ws[kProjMaxCz][8];
+    __shared__ float bs[8];
+    const int L = p.L, ngroups = p.C / 8, Cz = p.Cz;
+    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
+    for (int i = threadIdx.x; i < Cz * 8; i += NT_ACT) ws[i >> 3][i & 7] = __ldg(p.w + (size_t)(i >> 3) * p.C + g * 8 + (i & 7));
+    if (threadIdx.x < 8) bs[threadIdx.x] = __ldg(p.bias + g * 8 + threadIdx.x);
+    __syncthreads();
+    const int t = -p.pad_l + blockIdx.x * NT_ACT + threadIdx.x;
+    if (t >= L + p.pad_r) return;
+    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
+    const long long row = ((long long)b * ngroups + g) * Lpad + p.pad_l + t;
+    float v[8];
+    if (t >= 0 && t < L) {
+#pragma unroll
+        for (int o = 0; o < 8; ++o) v[o] = bs[o];
+        const float* zc = p.z + (long long)b * Cz * L + t;
+        for (int k = 0; k < Cz; ++k) {
+            const float zk = __ldg(zc + (long long)k * L);
+            const float4 w0 = *reinterpret_cast<const float4*>(&ws[k][0]);
+            const float4 w1 = *reinterpret_cast<const float4*>(&ws[k][4]);
+            v[0] = fmaf(w0.x, zk, v[0]);
+            v[1] = fmaf(w0.y, zk, v[1]);
+            v[2] = fmaf(w0.z, zk, v[2]);
+            v[3] = fmaf(w0.w, zk, v[3]);
+            v[4] = fmaf(w1.x, zk, v[4]);
+            v[5] = fmaf(w1.y, zk, v[5]);
+            v[6] = fmaf(w1.z, zk, v[6]);
+            v[7] = fmaf(w1.w, zk, v[7]);
+        }
+    } else {
+#pragma unroll
+        for (int o = 0; o < 8; ++o) v[o] = 0.f;   // the conv's zero padding
+    }
+    uint4 hv, lv;
+    split2(v[0], v[1], &hv.x, &lv.x);
+    split2(v[2], v[3], &hv.y, &lv.y);
+    split2(v[4], v[5], &hv.z, &lv.z);
+    split2(v[6], v[7], &hv.w, &lv.w);
+    reinterpret_cast<uint4*>(p.a_hi)[row] = hv;
+    reinterpret_cast<uint4*>(p.a_lo)[row] = lv;
+}
+
+// grid: x = output tiles of TT - (K - 1) samples, y = B.  Warp c stages the mean input window of
+// channel c, forms its 512 activation values of rows [t0 - pad, t0 - pad + 512) with the same
+// lane routine as k_act_split, and parks them in shared memory (zero outside [0, L): the conv's
+// padding); then every thread forms up to two outputs from the 8 x K window.
+__global__ void __launch_bounds__(NT_ACT) k_post_act(const PostParams p) {
+    __shared__ __align__(16) float xsb[8 * XF_P];
+    __shared__ __align__(16) float arow[8][TT];
+    __shared__ float wsh[8 * kPostMaxK];
+    const int L = p.L, K = p.K, TO = TT - (K - 1);
+    const int b = blockIdx.y;
+    const int t0 = blockIdx.x * TO;
+    const int tw = t0 - p.pad;                      // first activation row of the block
+    const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 8 * K; i += NT_ACT) wsh[i] = __ldg(p.w + i);
+    float* xs = xsb + c * XF_P;
+    const long long rb = ((long long)b * 8 + c) * L;
+    const bool edge = !(tw >= 8 && tw + TT + 8 <= L);
+    // mean of the three block outputs over x[tw - 8, tw + TT + 8), replicate-clamped at the ends
+    for (int i = lane; i < XF; i += 32) {
+        const long long g = rb + clampi(tw - 8 + i, 0, L - 1);
+        xs[skew(i)] = (__ldg(p.x0 + g) + __ldg(p.x1 + g) + __ldg(p.x2 + g)) / 3.0f;
+    }
+    __syncwarp();
+    const float al = __ldg(p.alpha + c), ib = __ldg(p.inv_beta + c);
+    float a[RUN];
+    if (edge) actm::act_lane<RUN, true>(p.filt, xs, al, ib, tw, L, a);
+    else actm::act_lane<RUN, false>(p.filt, xs, al, ib, tw, L, a);
+#pragma unroll
+    for (int k = 0; k < RUN; ++k) {
+        const int t = tw + RUN * lane + k;
+        arow[c][RUN * lane + k] = (t >= 0 && t < L) ? a[k] : 0.f;
+    }
+    __syncthreads();
+    const float bo = p.bias ? __ldg(p.bias) : 0.f;
+    if (K == 7) {
+        // two adjacent outputs per thread share 8 window values per channel
+        const int q = 2 * tid;
+        if (q < TO && t0 + q < L) {
+            float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float xa[8];
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const float2 v = *reinterpret_cast<const float2*>(&arow[cc][q + j]);
+                    xa[j] = v.x;
+                    xa[j + 1] = v.y;
+                }
+#pragma unroll
+                for (int j = 0; j < 7; ++j) {
+                    const float wv = wsh[cc * 7 + j];
+                    y0 = fmaf(wv, xa[j], y0);
+                    y1 = fmaf(wv, xa[j + 1], y1);
+                }
+            }
+            y0 += bo;
+            y1 += bo;
+            if (p.clamp) {   // NaN passes through
+                y0 = (y0 < -1.f) ? -1.f : ((y0 > 1.f) ? 1.f : y0);
+                y1 = (y1 < -1.f) ? -1.f : ((y1 > 1.f) ? 1.f : y1);
+            }
+            p.out[(long long)b * L + t0 + q] = y0;
+            if (q + 1 < TO && t0 + q + 1 < L) p.out[(long long)b * L + t0 + q + 1] = y1;
+        }
+    } else {
+        for (int q = tid; q < TO; q += NT_ACT) {
+            const int t = t0 + q;
+            if (t >= L) break;
+            float y = 0.f;
+            for (int cc = 0; cc < 8; ++cc)
+                for (int j = 0; j < K; ++j) y = fmaf(wsh[cc * K + j], arow[cc][q + j], y);
+            y += bo;
+            if (p.clamp) y = (y < -1.f) ? -1.f : ((y > 1.f) ? 1.f : y);   // NaN passes through
+            p.out[(long long)b * L + t] = y;
+        }
+    }
+}
+
 }  // namespace
+
+int launch_post_act(const PostParams& p, cudaStream_t s) {
+    if (p.L < 1 || p.B < 1 || p.K < 1 || p.K > kPostMaxK || p.pad < 0 || p.pad > p.K - 1 || !p.x0 || !p.x1 ||
+        !p.x2 || !p.w || !p.out)
+        return -1;
+    const int TO = TT - (p.K - 1);
+    dim3 grid((p.L + TO - 1) / TO, p.B);
+    k_post_act<<<grid, NT_ACT, 0, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
+
+int launch_proj_split(const ProjSplitParams& p, cudaStream_t s) {
+    if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0 || p.Cz < 1 || p.Cz > kProjMaxCz || !p.z || !p.w ||
+        !p.bias)
+        return -1;
+    const int total = p.L + p.pad_l + p.pad_r;
+    dim3 grid((total + NT_ACT - 1) / NT_ACT, p.B * (p.C / 8));
+    k_proj_split<<<grid, NT_ACT, 0, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
 
 int launch_split_rows(const SplitParams& p, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0 || !p.x0) return -1;

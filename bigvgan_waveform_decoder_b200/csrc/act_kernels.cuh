@@ -38,5 +38,38 @@ int launch_split_rows(const SplitParams& p, cudaStream_t s);
 // of kernels launched or -1.
 int launch_act_split(const ActParams& p, int njobs, cudaStream_t s);
 
+// dec_in_proj (a 1x1 conv, Cz -> C) fused into the head/tail split of its output, which is
+// conv_pre's A operand: h[c, t] = bias[c] + sum_k w[k, c] z[k, t], written as rows of 8
+// channels like launch_split_rows (h itself is never stored).
+struct ProjSplitParams {
+    const float* z;         // [B, Cz, L] latents
+    const float* w;         // [Cz, C] folded 1x1 weights
+    const float* bias;      // [C]
+    void* a_hi;             // [B, C/8, pad_l + L + pad_r] rows of 8 bf16 (heads)
+    void* a_lo;             // same shape (tails)
+    int Cz, C, L, B;
+    int pad_l, pad_r;
+};
+constexpr int kProjMaxCz = 64;   // latent channels the fused projection accepts
+int launch_proj_split(const ProjSplitParams& p, cudaStream_t s);
+
+// The decoder's tail in one kernel: the mean of the last stage's three block outputs, the
+// anti-aliased SnakeBeta (activation_post), the K-tap conv_post to one channel, its bias and
+// the clamp to [-1, 1].  Exactly 8 input channels (one warp each).
+struct PostParams {
+    const float* x0;        // [B, 8, L] block outputs
+    const float* x1;
+    const float* x2;
+    const float* alpha;     // [8]
+    const float* inv_beta;  // [8]
+    const float* w;         // [8, K] folded conv_post weights
+    const float* bias;      // [1] or null
+    float* out;             // [B, 1, L]
+    int L, B, K, pad;
+    int clamp;              // 1: clamp to [-1, 1] (NaN passes through)
+    ActFilter filt;
+};
+constexpr int kPostMaxK = 15;
+int launch_post_act(const PostParams& p, cudaStream_t s);
 
 }  // namespace mh3a

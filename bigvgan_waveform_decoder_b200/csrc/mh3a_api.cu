@@ -404,6 +404,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
     h->nseg = 0;
     mh3a_status st = record(h, s);
     if (st) return st;
+    const bool fused_proj = h->pre_tc && c.latent_channels <= kProjMaxCz;
     // dec_in_proj (denormalisation folded in)
     {
         ConvParams p{};
@@ -418,7 +419,28 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = 1;
         p.job[0].dil = 1;
         p.job[0].pad = 0;
-        if ((st = counted(h, launch_conv1x1(p, s)))) return st;
+        if (fused_proj) {
+            // the projection goes straight into conv_pre's head/tail operand rows
+            if ((long long)B * c.latent_dim * ((long long)N + kApadL + kApadR) > h->a_cap) {
+                g_last_error = "batch too large for the tensor-core operand buffers (B > max_batch)";
+                return MH3A_ERR_SHAPE;
+            }
+            ProjSplitParams pp{};
+            pp.z = lat;
+            pp.w = h->in_proj.w;
+            pp.bias = h->in_proj.b;
+            pp.a_hi = h->A_hi[0];
+            pp.a_lo = h->A_lo[0];
+            pp.Cz = c.latent_channels;
+            pp.C = c.latent_dim;
+            pp.L = N;
+            pp.B = B;
+            pp.pad_l = kApadL;
+            pp.pad_r = kApadR;
+            if ((st = counted(h, launch_proj_split(pp, s)))) return st;
+        } else {
+            if ((st = counted(h, launch_conv1x1(p, s)))) return st;
+        }
         if ((st = record(h, s))) return st;
     }
     // conv_pre
@@ -437,8 +459,9 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].pad = 3;
         int n;
         if (h->pre_tc) {
-            // split the input into head/tail rows once, then the persistent tensor-core GEMM
-            if ((st = split_to_a(h, h->buf_in, nullptr, nullptr, c.latent_dim, N, B, s))) return st;
+            // the input as head/tail rows (already written by the fused projection, or split
+            // here), then the persistent tensor-core GEMM
+            if (!fused_proj && (st = split_to_a(h, h->buf_in, nullptr, nullptr, c.latent_dim, N, B, s))) return st;
             n = launch_conv_pre_gemm(p, h->tc[0], h->A_hi[0], h->A_lo[0], kApadL, (long long)N + kApadL + kApadR,
                                      pre_parts(h), s, h->dev_err, h->dev_err + 16);
         } else {
@@ -510,7 +533,26 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         p.job[0].K = h->post.k;
         p.job[0].dil = 1;
         p.job[0].pad = 3;
-        if ((st = counted(h, launch_conv_simt(p, 1, true, true, s)))) return st;
+        if (c.precision == MH3A_BF16X3 && C == 8 && c.n_resblocks == 3) {
+            PostParams pp{};
+            pp.x0 = h->X[0];
+            pp.x1 = h->X[1];
+            pp.x2 = h->X[2];
+            pp.alpha = h->act_post.alpha;
+            pp.inv_beta = h->act_post.inv_beta;
+            pp.w = h->post.w;
+            pp.bias = h->post.b;
+            pp.out = out;
+            pp.L = L;
+            pp.B = B;
+            pp.K = h->post.k;
+            pp.pad = 3;
+            pp.clamp = p.clamp;
+            pp.filt = h->filt;
+            if ((st = counted(h, launch_post_act(pp, s)))) return st;
+        } else {
+            if ((st = counted(h, launch_conv_simt(p, 1, true, true, s)))) return st;
+        }
         if ((st = record(h, s))) return st;
     }
     return MH3A_OK;
