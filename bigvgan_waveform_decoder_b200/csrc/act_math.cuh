@@ -29,20 +29,13 @@ __device__ __forceinline__ int skew(int i) { return i + ((i >> 4) << 2); }
 // skewed size of a window of n floats
 __host__ __device__ constexpr int skewed(int n) { return n + n / 16 * 4 + 4; }
 
-// sin^2(alpha u): Cody-Waite reduction modulo pi, then the hardware sine on [-pi/2, pi/2]
-// (absolute error near 2^-21, far below the 3xBF16 operand error).
-// The nearest integer k = rint(v / pi) is formed by adding and subtracting 1.5 * 2^23 in
-// round-to-nearest fp32 arithmetic, exact for |v / pi| < 2^22.
+// sin^2(alpha u) with the hardware sine.  Its argument error grows with |alpha u| as the fp32
+// rounding of the product alpha u itself does (about |alpha u| 2^-24), so reducing the phase
+// modulo pi first would not make the result more accurate.  Relative to the SnakeBeta output
+// (of magnitude about |u|) both stay far below the 3xBF16 operand error (2^-17); the parity
+// tests bound the end-to-end effect.
 __device__ __forceinline__ float sin_sq_fast(float alpha, float u) {
-    const float kInvPi = 0.318309886183790671538f;
-    const float kPiHi = 3.14159274101257324219f;
-    const float kPiLo = -8.74227800037248297e-08f;
-    const float kRound = 12582912.0f;  // 1.5 * 2^23
-    const float v = alpha * u;
-    const float k = __fsub_rn(__fmaf_rn(v, kInvPi, kRound), kRound);
-    float r = fmaf(-k, kPiHi, v);
-    r = fmaf(-k, kPiLo, r);
-    const float s = __sinf(r);
+    const float s = __sinf(alpha * u);
     return s * s;
 }
 
