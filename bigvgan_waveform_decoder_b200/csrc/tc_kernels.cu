@@ -88,6 +88,11 @@ __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? l
 // each core column's head rows directly followed by its tail rows.
 __host__ __device__ constexpr bool interleaved_b(int NT, int R) { return R == 1 && NT <= 64; }
 
+// Upsampler rates whose taps are grouped by input row offset (one MMA over all phases per
+// group).  At rate 2 a group holds at most two taps, so the zero rows would cost what the wider
+// MMA saves.
+__host__ __device__ constexpr bool convt_grouped(int R) { return R > 2; }
+
 __device__ __forceinline__ void prod_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NPROD) : "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
@@ -537,7 +542,10 @@ __device__ __forceinline__ void add_res_group(float (&acc)[N], const float (&rq)
 // zero block stands in for the tap past the last one).
 // R > 1: the polyphase transposed conv (upsampler).  Rows are input samples u; tap j reads the
 // window at row offset tap_row[j] and accumulates into the region of its output phase
-// tap_phase[j]; the epilogue writes phase phi of row u to output sample R u + phi.  A pass is
+// tap_phase[j]; the epilogue writes phase phi of row u to output sample R u + phi.  With
+// GRP (R > 2) a unit is instead a group of taps sharing one row offset: its weight block holds
+// all R phases (zero rows where the group has no tap), so one MMA of N = R NT covers every
+// phase region and the group's first unit initialises all of them.  A pass is
 // then one whole chunk, so that the first tap of every phase (j < R) starts its region.
 template <int MT, int NT, int KGT, int EW, int R>
 __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
@@ -550,7 +558,9 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
     static_assert(EW == 8 || EW == 16, "epilogue warps");
     static_assert((4 * MT * NT / EW) % 16 == 0 && 4 * MT * NT / EW <= NT, "epilogue column split");
     constexpr int BG = (KGT == 1) ? 2 : KGT;
-    constexpr int TAPB = 2 * BG * NT * 16;
+    constexpr bool GRP = convt_grouped(R);                 // units are row-offset groups
+    constexpr int BROWS = GRP ? R * NT : NT;                // B rows per core column of a unit
+    constexpr int TAPB = 2 * BG * BROWS * 16;
     constexpr int CW = 4 * MT * NT / EW;                // accumulator columns per epilogue warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Cin = p.Cin, Cout = p.Cout, L = p.L;
@@ -607,9 +617,9 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         // warp-uniform; one elected lane issues each group of three MMAs and each commit.
         // Descriptors are built once per ring slot and advanced by adding 16-byte offsets to
         // their low word (the start-address field).
-        constexpr uint32_t idesc = ptx::idesc_bf16(128, NT);
+        constexpr uint32_t idesc = ptx::idesc_bf16(128, BROWS);
         constexpr uint32_t idesc_2n = ptx::idesc_bf16(128, ILV ? 2 * NT : NT);
-        constexpr uint32_t b_lbo = (ILV ? 2 * NT : NT) * 16;   // bytes between core columns
+        constexpr uint32_t b_lbo = (ILV ? 2 * NT : BROWS) * 16;   // bytes between core columns
         constexpr int KK = (KGT == 1) ? 1 : KGT / 2;   // K-steps per tap unit
         const uint32_t a_smem = ptx::smem_u32(As), b_smem = ptx::smem_u32(Bs);
         bool ok = *abort_flag == 0;
@@ -650,7 +660,10 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     uint32_t dbase = tmem + (uint32_t)(buf * PS_BUFCOLS);
                     uint32_t arow = ashift;
                     bool first = upass == 0;
-                    if (R > 1) {
+                    if (GRP) {
+                        arow = (uint32_t)J.tap_row[unit];
+                        first = unit == 0;
+                    } else if (R > 1) {
                         arow = (uint32_t)J.tap_row[unit];
                         dbase += (uint32_t)(J.tap_phase[unit] * NT);
                         first = unit < R;
@@ -669,8 +682,8 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                                                      ptx::desc64(a + (uint32_t)(KGT * RS)), ptx::desc64(bk), idesc_2n,
                                                      idesc, acc);
                             } else {
-                                const uint32_t bhk = bh + (uint32_t)(2 * kk * NT);
-                                const uint32_t blk = bhk + (uint32_t)(BG * NT);
+                                const uint32_t bhk = bh + (uint32_t)(2 * kk * BROWS);
+                                const uint32_t blk = bhk + (uint32_t)(BG * BROWS);
                                 ptx::mma3_bf16_elect(d, ptx::desc64(a), ptx::desc64(a + (uint32_t)(KGT * RS)),
                                                      ptx::desc64(bhk), ptx::desc64(blk), idesc, acc);
                             }
@@ -708,7 +721,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
     } else if (warp == 1) {
         // ---------------------------------------------------------------- A and B loader
         if (lane == 0) {
-            const size_t unit_elems = (size_t)2 * BG * NT * 8;
+            const size_t unit_elems = (size_t)2 * BG * BROWS * 8;
             bool ok = *abort_flag == 0;
             int ia = 0, ib = 0;
             bool drained = false;   // the scheduler handed this CTA its end marker
@@ -1026,9 +1039,11 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
             return -1;
         if (R > 1)
             for (int k = 0; k < J.K; ++k)
-                if (J.tap_phase[k] < 0 || J.tap_phase[k] >= R || J.tap_row[k] < 0 || J.tap_row[k] > J.span) return -1;
+                if (J.tap_row[k] < 0 || J.tap_row[k] > J.span ||
+                    (!convt_grouped(R) && (J.tap_phase[k] < 0 || J.tap_phase[k] >= R)))
+                    return -1;
     }
-    constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * NT * 16;
+    constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * (convt_grouped(R) ? R * NT : NT) * 16;
     p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));   // weight copies of about 16 KB
     PsSched sc{};
     sc.n_ot = (p.Cout + NT - 1) / NT;
@@ -1128,6 +1143,65 @@ void pack_blocks(W w, int Cout, int Cin, int K, int NT, int KGT, bool interleave
     out->k = K;
 }
 
+// Row-offset groups of a polyphase transposed conv (rate r <= 8, K <= 16 taps, padding pad):
+// tap j serves output phase (j - pad) mod r and reads input row u + (phase + pad - j) / r, so
+// two taps of one phase never share a row offset.  Groups are the distinct offsets in
+// increasing order; tap[g][phase] is the group's tap of that phase, or -1.
+struct ConvtGroups {
+    int n = 0;
+    int shift[16];
+    int tap[16][8];
+};
+
+ConvtGroups convt_groups(int K, int r, int pad) {
+    ConvtGroups G;
+    int sh[16];
+    for (int j = 0; j < K; ++j) {
+        const int phase = ((j - pad) % r + r) % r;
+        sh[j] = (phase + pad - j) / r;   // exact: phase + pad - j is a multiple of r
+    }
+    for (int v = -16; v <= 16; ++v) {
+        bool any = false;
+        for (int j = 0; j < K; ++j) any = any || sh[j] == v;
+        if (!any) continue;
+        G.shift[G.n] = v;
+        for (int ph = 0; ph < 8; ++ph) G.tap[G.n][ph] = -1;
+        for (int j = 0; j < K; ++j)
+            if (sh[j] == v) G.tap[G.n][((j - pad) % r + r) % r] = j;
+        ++G.n;
+    }
+    return G;
+}
+
+// Upsampler operand blocks with grouped units: [o_tile][chunk][group][part][core col]
+// [phase][row o][8 channels], the rows of a phase without a tap in the group zero.
+void pack_convt_grouped(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, int NT, int KGT,
+                        TcConv* out) {
+    const ConvtGroups G = convt_groups(K, r, (K - r) / 2);
+    const int kc = 8 * KGT, ntiles = (Cout + NT - 1) / NT, nchunks = Cin / kc;
+    const size_t n = (size_t)ntiles * nchunks * G.n * 2 * KGT * r * NT * 8;
+    std::vector<uint16_t> buf(n);
+    size_t pos = 0;
+    for (int ot = 0; ot < ntiles; ++ot)
+        for (int chk = 0; chk < nchunks; ++chk)
+            for (int g = 0; g < G.n; ++g)
+                for (int part = 0; part < 2; ++part)
+                    for (int col = 0; col < KGT; ++col)
+                        for (int ph = 0; ph < r; ++ph)
+                            for (int o = 0; o < NT; ++o)
+                                for (int e = 0; e < 8; ++e) {
+                                    const int oo = ot * NT + o, cc = chk * kc + col * 8 + e, tap = G.tap[g][ph];
+                                    const float v = (tap >= 0 && oo < Cout) ? w_iok[((size_t)cc * Cout + oo) * K + tap] : 0.f;
+                                    const uint16_t hb = bf16_bits_rn(v);
+                                    buf[pos++] = part == 0 ? hb : bf16_bits_rn(v - bf16_value(hb));
+                                }
+    out->staging.assign((n + 1) / 2, 0.f);
+    std::memcpy(out->staging.data(), buf.data(), n * sizeof(uint16_t));
+    out->cout = Cout;
+    out->cin = Cin;
+    out->k = K;
+}
+
 TcJob make_job(const ConvJob& J, const TcConv& tw) {
     TcJob T{};
     T.x0 = J.x0;
@@ -1187,6 +1261,10 @@ void prepare_tc_pre(const std::vector<float>& w, int O, int I, int k, TcStageWei
 }
 
 void prepare_tc_convt(const std::vector<float>& w_iok, int Cin, int Cout, int K, int r, TcConv* out) {
+    if (convt_grouped(r)) {
+        pack_convt_grouped(w_iok, Cin, Cout, K, r, ntile_convt(Cout, r), kgt_convt(Cin), out);
+        return;
+    }
     pack_blocks([&](int o, int c, int tap) { return w_iok[((size_t)c * Cout + o) * K + tap]; }, Cout, Cin, K,
                 ntile_convt(Cout, r), kgt_convt(Cin), interleaved_b(ntile_convt(Cout, r), r), out);
 }
@@ -1313,13 +1391,19 @@ int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void*
         smax = std::max(smax, sh[j]);
     }
     for (int j = 0; j < q.K; ++j) G.tap_row[j] = (int8_t)(sh[j] - smin);
+    G.K = q.K;
+    if (convt_grouped(q.r)) {
+        // units are the row-offset groups, in the packer's order
+        const ConvtGroups CG = convt_groups(q.K, q.r, q.pad);
+        for (int g = 0; g < CG.n; ++g) G.tap_row[g] = (int8_t)(CG.shift[g] - smin);
+        G.K = CG.n;
+    }
     G.a_hi = static_cast<const uint8_t*>(a_hi);
     G.a_lo = static_cast<const uint8_t*>(a_lo);
     G.w = reinterpret_cast<const uint16_t*>(w.ups.dev);
     G.bias = q.bias;
     G.res = nullptr;
     G.out = q.out;
-    G.K = q.K;
     G.dil = 1;
     G.pad = -smin;
     G.span = smax - smin;
