@@ -140,29 +140,26 @@ __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
     }
 }
 
-// Plain head/tail split (no activation) into the same row layout, of x0, of the mean
-// (x0 + x1 + x2) / 3 of three block outputs, or of the sum of four partial outputs.  grid: x = row tiles of NT_ACT, y = B * C / 8.
-__global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
-    const int L = p.L, ngroups = p.C / 8;
-    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
-    const int t = -p.pad_l + blockIdx.x * NT_ACT + threadIdx.x;
-    if (t >= L + p.pad_r) return;
-    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
-    const long long row = ((long long)b * ngroups + g) * Lpad + p.pad_l + t;
-    float v[8];
-    if (t >= 0 && t < L) {
-        const long long base = ((long long)b * p.C + g * 8) * L + t;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const long long i = base + (long long)c * L;
-            if (p.x3) v[c] = ((__ldg(p.x0 + i) + __ldg(p.x1 + i)) + __ldg(p.x2 + i)) + __ldg(p.x3 + i);
-            else if (p.x1) v[c] = (__ldg(p.x0 + i) + __ldg(p.x1 + i) + __ldg(p.x2 + i)) / 3.0f;
-            else v[c] = __ldg(p.x0 + i);
-        }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = 0.f;
+// Input value of channel row `ci` (index into [B, C, L]) in the form the split takes.
+__device__ __forceinline__ float split_in(const SplitParams& p, long long ci) {
+    if (p.x3) return ((__ldg(p.x0 + ci) + __ldg(p.x1 + ci)) + __ldg(p.x2 + ci)) + __ldg(p.x3 + ci);
+    if (p.x1) return (__ldg(p.x0 + ci) + __ldg(p.x1 + ci) + __ldg(p.x2 + ci)) * (1.0f / 3.0f);
+    return __ldg(p.x0 + ci);
+}
+
+__device__ __forceinline__ float2 split_in2(const SplitParams& p, long long ci) {
+    const float2 a = __ldg(reinterpret_cast<const float2*>(p.x0 + ci));
+    if (!p.x1) return a;
+    const float2 b = __ldg(reinterpret_cast<const float2*>(p.x1 + ci));
+    const float2 c = __ldg(reinterpret_cast<const float2*>(p.x2 + ci));
+    if (p.x3) {
+        const float2 d = __ldg(reinterpret_cast<const float2*>(p.x3 + ci));
+        return make_float2(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y);
     }
+    return make_float2((a.x + b.x + c.x) * (1.0f / 3.0f), (a.y + b.y + c.y) * (1.0f / 3.0f));
+}
+
+__device__ __forceinline__ void store_row(const SplitParams& p, long long row, const float (&v)[8]) {
     uint4 hv, lv;
     split2(v[0], v[1], &hv.x, &lv.x);
     split2(v[2], v[3], &hv.y, &lv.y);
@@ -170,6 +167,40 @@ __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
     split2(v[6], v[7], &hv.w, &lv.w);
     reinterpret_cast<uint4*>(p.a_hi)[row] = hv;
     reinterpret_cast<uint4*>(p.a_lo)[row] = lv;
+}
+
+// Plain head/tail split (no activation) into the same row layout, of x0, of the mean
+// (x0 + x1 + x2) / 3 of three block outputs, or of the sum of four partial outputs.  grid: x =
+// tiles of 2 NT_ACT rows (two adjacent rows per thread, read as float2 where both lie inside an
+// even-length sequence), y = B * C / 8.
+__global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
+    const int L = p.L, ngroups = p.C / 8;
+    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
+    const int t = -p.pad_l + 2 * (blockIdx.x * NT_ACT + threadIdx.x);   // the thread's first row
+    if (t >= L + p.pad_r) return;
+    const long long Lpad = (long long)L + p.pad_l + p.pad_r;
+    const long long row = ((long long)b * ngroups + g) * Lpad + p.pad_l + t;
+    const long long base = ((long long)b * p.C + g * 8) * L;
+    const bool second = t + 1 < L + p.pad_r;
+    float v0[8], v1[8];
+    const uintptr_t align = reinterpret_cast<uintptr_t>(p.x0) | reinterpret_cast<uintptr_t>(p.x1) |
+                            reinterpret_cast<uintptr_t>(p.x2) | reinterpret_cast<uintptr_t>(p.x3);
+    if ((L % 2 == 0) && (p.pad_l % 2 == 0) && (align & 7) == 0 && t >= 0 && t + 1 < L) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float2 v = split_in2(p, base + (long long)c * L + t);
+            v0[c] = v.x;
+            v1[c] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            v0[c] = (t >= 0 && t < L) ? split_in(p, base + (long long)c * L + t) : 0.f;
+            v1[c] = (t + 1 >= 0 && t + 1 < L) ? split_in(p, base + (long long)c * L + t + 1) : 0.f;
+        }
+    }
+    store_row(p, row, v0);
+    if (second) store_row(p, row + 1, v1);
 }
 
 // grid: x = row tiles of NT_ACT, y = B * C / 8.  The group's 8 x Cz weights and 8 biases sit in
@@ -321,7 +352,7 @@ int launch_split_rows(const SplitParams& p, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0 || !p.x0) return -1;
     if ((p.x1 == nullptr) != (p.x2 == nullptr) || (p.x3 && !p.x1)) return -1;
     const int total = p.L + p.pad_l + p.pad_r;
-    dim3 grid((total + NT_ACT - 1) / NT_ACT, p.B * (p.C / 8));
+    dim3 grid((total + 2 * NT_ACT - 1) / (2 * NT_ACT), p.B * (p.C / 8));
     k_split_rows<<<grid, NT_ACT, 0, s>>>(p);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
