@@ -116,6 +116,8 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
 
 // grid: x = row tiles over [-pad_l, L + pad_r), y = B * C / 8 (item, group), z = job
 __global__ void __launch_bounds__(NT_ACT) k_act_split(const ActParams p) {
+    ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
+    ptx::grid_dep_launch();
     __shared__ __align__(16) float buf[SMEM_FLOATS];
     const ActJob& J = p.job[blockIdx.z];
     const int L = p.L;
@@ -174,6 +176,8 @@ __device__ __forceinline__ void store_row(const SplitParams& p, long long row, c
 // tiles of 2 NT_ACT rows (two adjacent rows per thread, read as float2 where both lie inside an
 // even-length sequence), y = B * C / 8.
 __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
+    ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
+    ptx::grid_dep_launch();
     const int L = p.L, ngroups = p.C / 8;
     const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
     const int t = -p.pad_l + 2 * (blockIdx.x * NT_ACT + threadIdx.x);   // the thread's first row
@@ -206,6 +210,8 @@ __global__ void __launch_bounds__(NT_ACT) k_split_rows(const SplitParams p) {
 // grid: x = row tiles of NT_ACT, y = B * C / 8.  The group's 8 x Cz weights and 8 biases sit in
 // shared memory (read back as broadcasts); every thread forms one row of 8 channels.
 __global__ void __launch_bounds__(NT_ACT) k_proj_split(const ProjSplitParams p) {
+    ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
+    ptx::grid_dep_launch();
     __shared__ __align__(16) float ws[kProjMaxCz][8];
     __shared__ float bs[8];
     const int L = p.L, ngroups = p.C / 8, Cz = p.Cz;
@@ -253,6 +259,8 @@ __global__ void __launch_bounds__(NT_ACT) k_proj_split(const ProjSplitParams p) 
 // lane routine as k_act_split, and parks them in shared memory (zero outside [0, L): the conv's
 // padding); then every thread forms up to two outputs from the 8 x K window.
 __global__ void __launch_bounds__(NT_ACT) k_post_act(const PostParams p) {
+    ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
+    ptx::grid_dep_launch();
     __shared__ __align__(16) float xsb[8 * XF_P];
     __shared__ __align__(16) float arow[8][TT];
     __shared__ float wsh[8 * kPostMaxK];
@@ -334,8 +342,7 @@ int launch_post_act(const PostParams& p, cudaStream_t s) {
         return -1;
     const int TO = TT - (p.K - 1);
     dim3 grid((p.L + TO - 1) / TO, p.B);
-    k_post_act<<<grid, NT_ACT, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+    return launch_dependent(k_post_act, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
 }
 
 int launch_proj_split(const ProjSplitParams& p, cudaStream_t s) {
@@ -344,8 +351,7 @@ int launch_proj_split(const ProjSplitParams& p, cudaStream_t s) {
         return -1;
     const int total = p.L + p.pad_l + p.pad_r;
     dim3 grid((total + NT_ACT - 1) / NT_ACT, p.B * (p.C / 8));
-    k_proj_split<<<grid, NT_ACT, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+    return launch_dependent(k_proj_split, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
 }
 
 int launch_split_rows(const SplitParams& p, cudaStream_t s) {
@@ -353,16 +359,14 @@ int launch_split_rows(const SplitParams& p, cudaStream_t s) {
     if ((p.x1 == nullptr) != (p.x2 == nullptr) || (p.x3 && !p.x1)) return -1;
     const int total = p.L + p.pad_l + p.pad_r;
     dim3 grid((total + 2 * NT_ACT - 1) / (2 * NT_ACT), p.B * (p.C / 8));
-    k_split_rows<<<grid, NT_ACT, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+    return launch_dependent(k_split_rows, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
 }
 
 int launch_act_split(const ActParams& p, int njobs, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0) return -1;
     const int total = p.L + p.pad_l + p.pad_r;
     dim3 grid((total + TT - 1) / TT, p.B * (p.C / 8), njobs);
-    k_act_split<<<grid, NT_ACT, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+    return launch_dependent(k_act_split, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
 }
 
 }  // namespace mh3a

@@ -3,12 +3,34 @@
 
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 #include "mh3a.h"  // include/ is on the include path
 
 namespace mh3a {
 
 constexpr int kFilterTaps = 12;  // activation filter length (ratio 2: 6 * ratio)
+
+// Launch with programmatic dependent launch allowed: the grid may be scheduled while the
+// previous kernel of the stream is still finishing.  Every kernel launched this way executes
+// griddepcontrol.wait (ptx::grid_dep_wait) before it reads or writes global memory, which
+// waits for the preceding grid to complete and its writes to be visible, so stream order of the
+// data is kept; only the launch and the block scheduling overlap the predecessor's tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Anti-aliased SnakeBeta filter taps: f (decimator) and 2 f (upsampler, gain = ratio).
 struct ActFilter {

@@ -550,6 +550,7 @@ __device__ __forceinline__ void add_res_group(float (&acc)[N], const float (&rq)
 template <int MT, int NT, int KGT, int EW, int R>
 __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    ptx::grid_dep_wait();   // launched as a programmatic dependent (see launch_dependent)
     constexpr bool ILV = interleaved_b(NT, R);            // two-MMA K-steps, head | cross columns
     constexpr int RSTR = ILV ? 2 * NT : R * NT;            // accumulator columns per M tile
     static_assert(MT * RSTR <= PS_BUFCOLS, "one accumulator buffer holds MT x RSTR columns");
@@ -922,6 +923,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             atomicExch(p.err, 7);
         }
     }
+    ptx::grid_dep_launch();   // every role is done: the next grid may be scheduled
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -1073,8 +1075,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     auto kern = k_gemm_ps<MT, NT, KGT, EW, R>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_req) != cudaSuccess) return -1;
     const int grid = std::min(sc.ntiles, nsm);
-    kern<<<grid, ps_threads(EW), smem_req, s>>>(p, sc, pl);
-    return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+    return launch_dependent(kern, dim3(grid), dim3(ps_threads(EW)), smem_req, s, p, sc, pl) == cudaSuccess ? 1 : -1;
 }
 
 int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
