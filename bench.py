@@ -285,6 +285,7 @@ def run_ours(args):
                        "pipe": "tensor" if sgm.tensor else "fp32"})
     dom = max(range(len(stages)), key=lambda i: stages[i]["ms"]) if stages else None
     roofline = None
+    roofline_act = None
     if dom is not None:
         sgm, ms = segs[dom], seg_ms[dom]
         launches_in_seg = 6 if sgm.name.startswith("amp") else 1
@@ -304,6 +305,16 @@ def run_ours(args):
                         "activation_kernel_ms_per_launch": act_launch_ms,
                         "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
                                       "bf16 products per fp32 product"}
+            # the same stage's activation kernel, the other half of every AMP layer: fp32 work
+            # (56 flops per output, the 2 sines per output run on the SFU and are not counted)
+            act_flops = sgm.act_flops / 6
+            act_achieved = act_flops / (act_launch_ms * 1e-3) / 1e12
+            roofline_act = {"bound": "alu", "achieved": act_achieved, "peak": p_fp32, "unit": "TFLOP/s",
+                            "frac": act_achieved / p_fp32, "traffic": None,
+                            "kernel": f"k_act_split ({sgm.name}, 3 residual blocks per launch)",
+                            "launch_ms": act_launch_ms, "launches_per_step": launches_in_seg,
+                            "flops_per_launch": act_flops,
+                            "peak_basis": f"148 SM x 128 fp32 lanes x 2 x {peaks['sm_max_mhz']} MHz"}
         elif sgm.tensor:
             achieved = sgm.conv_flops / (ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
@@ -330,6 +341,7 @@ def run_ours(args):
                    "global_batch": B * world, "latent_frames": N, "replicas": world,
                    "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)"},
         "roofline": roofline,
+        "roofline_activation": roofline_act,
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": int(z.nbytes), "d2h_bytes_per_step": int(yp.numel() * 4)},
         "gpu_launches": launches,
