@@ -90,3 +90,22 @@ def test_amp_stage0_full_size_sampled(dev):
             khi = hi if hi == L else hi - RF_STAGE
             check(y[b, :, klo:khi], ref[:, klo - lo:khi - lo], Bd.MH3A_BF16X3,
                   f"AMP stage 0 item {b} samples {klo}-{khi}")
+
+
+@pytest.mark.parametrize("B,N", [(2, 7), (1, 1)])
+def test_decode_bench_arch_short_odd_lengths(dev, B, N):
+    """The bench architecture at short, odd latent lengths, compared over the whole output.  Every
+    tile of every tensor-core kernel is a ragged edge tile here: the split-K conv_pre and the
+    projection fused into its operand split, odd-length upsampler input splits (no paired
+    loads), the grouped rate-5 upsamplers and the fused activation_post + conv_post."""
+    arch = S.Arch()
+    w = S.workload_weights(3, arch)
+    z = S.make_latents(B, N, arch.latent_channels, 11)
+    d = Bd.Decoder(arch, w, precision=Bd.MH3A_BF16X3, max_batch=B, max_frames=N, no_clamp=True)
+    y = d.decode(torch.from_numpy(z).to(dev)).cpu().numpy()
+    d.check_device_error()
+    d.close()
+    assert y.shape == (B, 1, HOP * N)
+    ref = oracle.decode(arch, w, z, clamp=False)
+    for b in range(B):
+        check(y[b, 0], ref[b, 0], Bd.MH3A_BF16X3, f"bench arch B={B} N={N} item {b}", waveform=True)
