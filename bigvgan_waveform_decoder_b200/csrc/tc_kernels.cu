@@ -830,7 +830,17 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             float acc[R * CW];
 #pragma unroll
             for (int c = 0; c < CW; ++c) acc[c] = 0.f;
-            if (!kSpread && has_res) {
+            // 16-column warps keep the residual apart and add it after the last pass, so that
+            // the first drain does not wait for the loads
+            constexpr bool kLate = R == 1 && CW == 16;
+            float rl[kLate ? CW : 1];
+            if constexpr (kLate) {
+                if (has_res) {
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) rl[c] = (NT > 16 || o_base + c < Cout) ? __ldg(rp + (long long)c * Lout) : 0.f;
+                }
+            }
+            if (!kLate && !kSpread && has_res) {
                 if (NT > 16 || o_base + CW <= Cout) {
 #pragma unroll
                     for (int c = 0; c < CW; ++c) acc[c] = __ldg(rp + (long long)c * Lout);
@@ -907,6 +917,12 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             if (!ok || *abort_flag) {
                 ok = false;
                 break;
+            }
+            if constexpr (kLate) {
+                if (has_res) {
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) acc[c] += rl[c];
+                }
             }
             if (t < L) {
 #pragma unroll
