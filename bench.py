@@ -47,7 +47,7 @@ GEMM_TILE = {512: "1, 256, 4, 8, 1", 256: "1, 256, 4, 8, 1", 128: "2, 128, 4, 8,
 # DRAM bytes (read + write) per launch of that GEMM kernel on this workload, keyed by (channels,
 # B * N), from one ncu capture (profiles/k_gemm_ps_stage1_B2_L10000.md); null when unmeasured
 # or when the kernel changed after the capture.
-GEMM_TRAFFIC = {(256, 800): 110.7e6}
+GEMM_TRAFFIC = {(256, 800): 110.4e6}
 UNIT = "audio-s/s"
 WORKLOAD = 3
 FLUSH_BYTES = 256 << 20
