@@ -75,6 +75,21 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: the replicas' job ends when the last one does."""
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, audio_s_per_step: float, max_ms: float) -> float:
+    """Whole-job audio-seconds per second: every rank decodes its own batch in every step."""
+    return world * steps * audio_s_per_step / (max_ms / 1e3)
+
+
 class Clocks:
     """nvidia-smi sampler of SM clock and throttle reasons while the timed region runs."""
 
@@ -254,12 +269,8 @@ def run_ours(args):
     dec.set_profiling(False)
     torch.cuda.synchronize()
 
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_max_ms = float(t.item())
-    value = world * args.steps * audio_s / (total_max_ms / 1e3)
+    total_max_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = job_throughput(world, args.steps, audio_s, total_max_ms)
 
     # end to end through the host-buffer entry point (pinned host memory)
     zp = torch.from_numpy(z).pin_memory()
@@ -275,10 +286,7 @@ def run_ours(args):
         ev1.record(stream)
         ev1.synchronize()
         e2e_ms.append(ev0.elapsed_time(ev1))
-    t = torch.tensor([sum(e2e_ms)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * args.steps * audio_s / (float(t.item()) / 1e3)
+    e2e_value = job_throughput(world, args.steps, audio_s, max_over_ranks(sum(e2e_ms), world, dev))
 
     # per-segment roofline
     segs = PM.segments(arch, B, N)
