@@ -13,12 +13,16 @@ around the timed region and in the max-over-ranks reduction of the timings.
 
 Timing: W untimed warm-up decodes, then K decodes, each bracketed by CUDA events on the
 launching stream; a 256 MiB buffer (> 126 MB L2) is rewritten between steps outside the events,
-so every step starts with a cold L2.  GPU clocks are sampled with nvidia-smi during the timed
-region.  Inside it, only the most expensive AMP stage carries CUDA events around its kernels
-(the roofline's per-launch times); the per-segment table comes from a few untimed decodes with
-segment events afterwards.  `e2e` repeats the measurement through mh3a_decode_host with pinned
-host buffers (host->device copy of the latents and device->host copy of the waveform inside the
-timing).
+so every step starts with a cold L2.  `ms_per_step` is the median step (the mean is reported
+beside it).  GPU clocks are sampled with nvidia-smi during the timed region.  The timed decodes
+carry no other events: the per-launch kernel times of the dominant AMP stage (the roofline) and
+the per-segment table come from untimed decodes afterwards, each with its own events.  `e2e`
+repeats the measurement through mh3a_decode_host with pinned host buffers (host->device copy of
+the latents and device->host copy of the waveform inside the timing).
+
+Two more workloads are reported as extra keys (the headline stays the 10 s stereo decode): the
+single AMP stage x [2, 512, 2000] through mh3a_amp_stage (`amp_stage`), and the batched 20 s
+decode B=16, N=800 with per-channel latent denormalisation (`batched_decode`).
 
 `--impl reference` times the fp64 CPU oracle (the correctness reference) on the host cores
 on a bounded sample of the same workload; under torchrun only rank 0 runs it.
@@ -48,6 +52,7 @@ GEMM_TILE = {512: "1, 256, 4, 8, 1", 256: "1, 256, 4, 8, 1", 128: "2, 128, 4, 8,
 # B * N), from one ncu capture (profiles/k_gemm_ps_stage1_B2_L10000.md); null when unmeasured
 # or when the kernel changed after the capture.
 GEMM_TRAFFIC = {(256, 800): 110.4e6}
+GEMM_TRAFFIC_SRC = "profiles/k_gemm_ps_stage1_B2_L10000.md"
 UNIT = "audio-s/s"
 WORKLOAD = 3
 FLUSH_BYTES = 256 << 20
@@ -61,10 +66,12 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--precision", choices=["bf16x3", "fp32"], default="bf16x3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-frames", type=int, default=40,
-                    help="latent frames of one batch item the CPU baseline decodes")
-    ap.add_argument("--ref-sample-frames", type=int, default=8,
-                    help="latent frames of one batch item per reference-arm step")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the single-stage and batched-decode figures")
+    ap.add_argument("--ref-sample-frames", type=int, default=200,
+                    help="latent frames of one batch item per reference-arm step; the oracle's "
+                         "fixed cost per batch item (its weight-norm folds) stays near 5 percent "
+                         "of a step at 200 frames")
     return ap.parse_args()
 
 
@@ -134,20 +141,20 @@ class Clocks:
                 "samples": len(rows), "reasons": sorted(reasons)}
 
 
-def cpu_baseline(frames: int) -> dict:
-    """The oracle as it stands, on one batch item of the workload, `frames` latents."""
+def cpu_baseline() -> dict:
+    """The oracle as it stands, on the whole workload: both items, all 400 latent frames."""
     import oracle
     from bigvgan_waveform_decoder_b200 import synthetic as S
 
     arch, w, z = S.workload_inputs(WORKLOAD)
-    zs = z[:1, :, :frames].copy()
+    B, _, N = z.shape
     t0 = time.perf_counter()
-    oracle.decode(arch, w, zs)
+    oracle.decode(arch, w, z)
     dt = time.perf_counter() - t0
-    audio_s = frames / 40.0
+    audio_s = B * N / 40.0
     return {"value": audio_s / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"1 batch item x {frames} latent frames ({audio_s:g} audio-s) of the "
-                      f"B=2 N=400 workload, fp64 oracle, {dt:.1f} s wall"}
+            "sample": f"B={B} N={N} in full ({audio_s:g} audio-s), fp64 oracle, one decode, "
+                      f"{dt:.1f} s wall"}
 
 
 def run_reference(args):
@@ -167,11 +174,12 @@ def run_reference(args):
         t0 = time.perf_counter()
         oracle.decode(arch, w, zs)
         times.append(time.perf_counter() - t0)
-    total = sum(times)
-    value = args.steps * audio_s / total
+    med = statistics.median(times)
+    value = audio_s / med
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * med,
+        "ms_per_step_mean": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": "decode B=2 N=400 (10 s stereo), sampled: 1 item x "
@@ -185,8 +193,76 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def timed_calls(fn, flush, steps: int, stream) -> list[float]:
+    """CUDA-event time (ms) of each of `steps` calls of fn on `stream`, L2 flushed before each
+    call outside its events."""
+    import torch
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for k in range(steps):
+        flush.fill_(float(k))
+        ev0.record(stream)
+        fn()
+        ev1.record(stream)
+        ev1.synchronize()
+        out.append(ev0.elapsed_time(ev1))
+    return out
+
+
+def extra_amp_stage(Bd, PM, peaks, p_tc, p_fp32, flush, stream, dev, steps: int) -> dict:
+    """The single-AMP-stage workload: x [2, 512, 2000] ~ N(0,1) and weights of seed 1, through
+    mh3a_amp_stage (the kernels the decode runs for its first AMP stage)."""
+    import torch
+    from bigvgan_waveform_decoder_b200 import synthetic as S
+
+    arch, w, xn = S.workload_inputs(1)
+    B, C, L = xn.shape
+    stage = S.WORKLOADS[1].stage
+    dec = Bd.Decoder(arch, w, precision=Bd.MH3A_BF16X3, max_batch=B,
+                     max_frames=-(-L // (arch.rates[0])))
+    x = torch.from_numpy(xn).to(dev)
+    out = torch.empty_like(x)
+    for _ in range(3):
+        dec.amp_stage(x, stage, out)
+    torch.cuda.synchronize()
+    ms = timed_calls(lambda: dec.amp_stage(x, stage, out), flush, steps, stream)
+    dec.check_device_error()
+    dec.close()
+    # x [2, 512, 2000] is exactly the decode's amp0 segment at B = 2, N = 400
+    seg = [sg for sg in PM.segments(arch, B, L // arch.rates[0]) if sg.name == "amp0"][0]
+    seg.tensor = True
+    roof = PM.roofline_time(seg, p_tc, p_fp32, peaks["hbm_gbs"]) * 1e3
+    med = statistics.median(ms)
+    return {"workload": f"AMP stage {stage}, x [{B}, {C}, {L}] (seed {S.WORKLOADS[1].seed})",
+            "ms": med, "conv_tflops": seg.conv_flops / (med * 1e-3) / 1e12, "roof_ms": roof,
+            "frac": roof / med, "calls": steps, "statistic": "median call",
+            "l2": "flushed between calls"}
+
+
+def extra_batched(arch_w, Bd, flush, stream, dev, steps: int) -> dict:
+    """The batched 20 s decode: B=16, N=800, per-channel latent denormalisation, seed 4."""
+    import torch
+    from bigvgan_waveform_decoder_b200 import synthetic as S
+
+    arch, w, z = arch_w
+    B, _, N = z.shape
+    dec = Bd.Decoder(arch, w, precision=Bd.MH3A_BF16X3, max_batch=B, max_frames=N)
+    x = torch.from_numpy(z).to(dev)
+    out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
+    for _ in range(2):
+        dec.decode(x, out)
+    torch.cuda.synchronize()
+    ms = timed_calls(lambda: dec.decode(x, out), flush, steps, stream)
+    dec.check_device_error()
+    dec.close()
+    med = statistics.median(ms)
+    return {"workload": f"decode B={B} N={N} (20 s, denormalised latents, seed 4)",
+            "value": B * N / 40.0 / (med * 1e-3), "unit": UNIT, "ms_per_step": med, "steps": steps,
+            "l2": "inputs and every stage tensor larger than L2; flushed between steps"}
+
+
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -212,54 +288,37 @@ def run_ours(args):
     flush = torch.empty(FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream()
     audio_s = B * N / 40.0
+    n_stages = len(arch.rates)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    dec.set_profiling(True)
     for _ in range(args.warmup):
         flush.fill_(1.0)
         dec.decode(x, out)
-    torch.cuda.synchronize()
-    # the dominant AMP stage of the warm-up decodes gets per-launch kernel events while timed
-    warm = dec.segment_times()
-    n_stages = len(arch.rates)
-    amp_ms = [warm[3 + 2 * i] if 3 + 2 * i < len(warm) else 0.0 for i in range(n_stages)]
-    kstage = max(range(n_stages), key=lambda i: amp_ms[i])
-    kstage = kstage if dec.stage_uses_tensor_cores(kstage) else -1
-    dec.set_kernel_profiling(kstage)
-    # the timed decodes carry no segment events (an event between two kernels keeps the second
-    # from being scheduled while the first finishes); only the dominant stage's kernel events
-    dec.set_profiling(False)
     barrier()
     torch.cuda.synchronize()
 
+    # ---- timed region: K decodes, nothing but the step events on the stream
     clocks = Clocks(local)
     clocks.start()
     launches0 = dec.launch_count()
-    step_ms, seg_sum = [], None
-    kern_sum = [[0.0, 0.0] for _ in range(n_stages)]   # per AMP stage: activation, GEMM ms
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for k in range(args.steps):
-        flush.fill_(float(k))
-        ev0.record(stream)
-        dec.decode(x, out)
-        ev1.record(stream)
-        ev1.synchronize()
-        step_ms.append(ev0.elapsed_time(ev1))
-        if kstage >= 0:
-            a_ms, g_ms = dec.stage_kernel_times(kstage)
-            kern_sum[kstage][0] += a_ms
-            kern_sum[kstage][1] += g_ms
+    step_ms = timed_calls(lambda: dec.decode(x, out), flush, args.steps, stream)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     launches = dec.launch_count() - launches0
     clk = clocks.stop()
-    dec.set_kernel_profiling(-1)
-    # per-segment times for the stage table: segment events on a few untimed decodes
-    n_seg = max(2, min(args.steps, 5))
+    dec.check_device_error()
+
+    med_ms = max_over_ranks(statistics.median(step_ms), world, dev)
+    value = job_throughput(world, 1, audio_s, med_ms)
+
+    # ---- untimed decodes with events: the per-segment table, then per-launch kernel times of
+    # the most expensive AMP stage (each event between two kernels costs a little overlap)
+    n_seg = 5
+    seg_sum = None
     dec.set_profiling(True)
     for k in range(n_seg):
         flush.fill_(float(k))
@@ -267,36 +326,38 @@ def run_ours(args):
         seg = dec.segment_times()
         seg_sum = seg if seg_sum is None else [a + b for a, b in zip(seg_sum, seg)]
     dec.set_profiling(False)
+    seg_ms = [t / n_seg for t in seg_sum]
+    amp_ms = [seg_ms[3 + 2 * i] for i in range(n_stages)]
+    kstage = max(range(n_stages), key=lambda i: amp_ms[i])
+    kern = [0.0, 0.0]
+    n_kern = 5
+    if dec.stage_uses_tensor_cores(kstage):
+        dec.set_kernel_profiling(kstage)
+        for k in range(n_kern):
+            flush.fill_(float(k))
+            dec.decode(x, out)
+            a_ms, g_ms = dec.stage_kernel_times(kstage)
+            kern[0] += a_ms
+            kern[1] += g_ms
+        dec.set_kernel_profiling(-1)
     torch.cuda.synchronize()
 
-    total_max_ms = max_over_ranks(sum(step_ms), world, dev)
-    value = job_throughput(world, args.steps, audio_s, total_max_ms)
-
-    # end to end through the host-buffer entry point (pinned host memory)
+    # ---- end to end through the host-buffer entry point (pinned host memory)
     zp = torch.from_numpy(z).pin_memory()
     yp = torch.empty((B, 1, dec.hop * N), dtype=torch.float32).pin_memory()
     for _ in range(args.warmup):
         dec.decode_host(zp, yp)
     barrier()
-    e2e_ms = []
-    for k in range(args.steps):
-        flush.fill_(float(k))
-        ev0.record(stream)
-        dec.decode_host(zp, yp)
-        ev1.record(stream)
-        ev1.synchronize()
-        e2e_ms.append(ev0.elapsed_time(ev1))
-    e2e_value = job_throughput(world, args.steps, audio_s, max_over_ranks(sum(e2e_ms), world, dev))
+    e2e_ms = timed_calls(lambda: dec.decode_host(zp, yp), flush, args.steps, stream)
+    e2e_value = job_throughput(world, 1, audio_s, max_over_ranks(statistics.median(e2e_ms), world, dev))
 
-    # per-segment roofline
+    # ---- per-segment roofline
     segs = PM.segments(arch, B, N)
     for i, sgm in enumerate(segs):
         sgm.tensor = dec.segment_uses_tensor_cores(i)
-    dec.check_device_error()
     peaks = PM.measured_peaks()
     p_fp32 = PM.fp32_peak_tflops(peaks["sm_max_mhz"])
     p_tc = peaks["bf16_tflops"] / 3.0
-    seg_ms = [s / n_seg for s in (seg_sum or [])]
     stages = []
     for sgm, ms in zip(segs, seg_ms):
         roof = PM.roofline_time(sgm, p_tc, p_fp32, peaks["hbm_gbs"]) * 1e3
@@ -304,63 +365,50 @@ def run_ours(args):
                        "frac": round(roof / ms, 4) if ms > 0 else None,
                        "tflops": round(sgm.flops / (ms * 1e-3) / 1e12, 2) if ms > 0 else None,
                        "pipe": "tensor" if sgm.tensor else "fp32"})
-    dom = max(range(len(stages)), key=lambda i: stages[i]["ms"]) if stages else None
+    sgm = segs[3 + 2 * kstage]
+    C = arch.decoder_dim >> (kstage + 1)
     roofline = None
     roofline_act = None
-    if dom is not None:
-        sgm, ms = segs[dom], seg_ms[dom]
-        launches_in_seg = 6 if sgm.name.startswith("amp") else 1
-        stage_i = int(sgm.name[3:]) if sgm.name.startswith("amp") else None
-        if sgm.tensor and stage_i is not None and kern_sum[stage_i][1] > 0:
-            # the stage's GEMM kernel alone: algorithmic flops of one launch (3 residual blocks)
-            # over its average launch duration, from the per-launch events of the timed steps
-            gemm_launch_ms = kern_sum[stage_i][1] / args.steps / 6
-            act_launch_ms = kern_sum[stage_i][0] / args.steps / 6
-            achieved = sgm.conv_flops / 6 / (gemm_launch_ms * 1e-3) / 1e12
-            C = arch.decoder_dim >> (stage_i + 1)
-            roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
-                        "frac": achieved / p_tc, "traffic": GEMM_TRAFFIC.get((C, B * N)),
-                        "kernel": f"k_gemm_ps<{GEMM_TILE.get(C, '?')}> ({sgm.name} conv, 3 residual blocks per launch)",
-                        "launch_ms": gemm_launch_ms, "launches_per_step": launches_in_seg,
-                        "flops_per_launch": sgm.conv_flops / 6,
-                        "activation_kernel_ms_per_launch": act_launch_ms,
-                        "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
-                                      "bf16 products per fp32 product"}
-            # the same stage's activation kernel, the other half of every AMP layer: fp32 work
-            # (56 flops per output, the 2 sines per output run on the SFU and are not counted)
-            act_flops = sgm.act_flops / 6
-            act_achieved = act_flops / (act_launch_ms * 1e-3) / 1e12
-            roofline_act = {"bound": "alu", "achieved": act_achieved, "peak": p_fp32, "unit": "TFLOP/s",
-                            "frac": act_achieved / p_fp32, "traffic": None,
-                            "kernel": f"k_act_split ({sgm.name}, 3 residual blocks per launch)",
-                            "launch_ms": act_launch_ms, "launches_per_step": launches_in_seg,
-                            "flops_per_launch": act_flops,
-                            "peak_basis": f"148 SM x 128 fp32 lanes x 2 x {peaks['sm_max_mhz']} MHz"}
-        elif sgm.tensor:
-            achieved = sgm.conv_flops / (ms * 1e-3) / 1e12
-            roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
-                        "frac": achieved / p_tc, "traffic": None,
-                        "kernel": f"{sgm.name} conv (segment)",
-                        "launches_per_step": launches_in_seg,
-                        "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
-                                      "bf16 products per fp32 product"}
-        else:
-            achieved = sgm.flops / (ms * 1e-3) / 1e12
-            roofline = {"bound": "alu", "achieved": achieved, "peak": p_fp32, "unit": "TFLOP/s",
-                        "frac": achieved / p_fp32, "traffic": None,
-                        "kernel": f"{sgm.name} fp32 conv+activation (3 residual blocks per launch)",
-                        "launches_per_step": launches_in_seg,
+    if kern[1] > 0:
+        # the stage's GEMM kernel alone: algorithmic flops of one launch (3 residual blocks)
+        # over its average launch duration
+        gemm_launch_ms = kern[1] / n_kern / 6
+        act_launch_ms = kern[0] / n_kern / 6
+        achieved = sgm.conv_flops / 6 / (gemm_launch_ms * 1e-3) / 1e12
+        traffic = GEMM_TRAFFIC.get((C, B * N))
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": p_tc, "unit": "TFLOP/s",
+                    "frac": achieved / p_tc, "traffic": traffic,
+                    "traffic_source": (f"{GEMM_TRAFFIC_SRC} (an earlier ncu capture of the same kernel "
+                                       "build, not measured in this run)") if traffic else None,
+                    "kernel": f"k_gemm_ps<{GEMM_TILE.get(C, '?')}> ({sgm.name} conv, 3 residual blocks per launch)",
+                    "launch_ms": gemm_launch_ms, "launches_per_step": 6,
+                    "flops_per_launch": sgm.conv_flops / 6,
+                    "activation_kernel_ms_per_launch": act_launch_ms,
+                    "timing": f"CUDA events around each launch, {n_kern} untimed decodes after the timed region",
+                    "peak_basis": f"bf16 burst {peaks['bf16_tflops']} ({peaks['source']}) / 3 "
+                                  "bf16 products per fp32 product"}
+        # the same stage's activation kernel, the other half of every AMP layer: fp32 work
+        # (56 flops per output; the 2 sines per output run on the SFU and are not counted)
+        act_flops = sgm.act_flops / 6
+        act_achieved = act_flops / (act_launch_ms * 1e-3) / 1e12
+        roofline_act = {"bound": "alu", "achieved": act_achieved, "peak": p_fp32, "unit": "TFLOP/s",
+                        "frac": act_achieved / p_fp32, "traffic": None,
+                        "kernel": f"k_act_split ({sgm.name}, 3 residual blocks per launch)",
+                        "launch_ms": act_launch_ms, "launches_per_step": 6,
+                        "flops_per_launch": act_flops,
                         "peak_basis": f"148 SM x 128 fp32 lanes x 2 x {peaks['sm_max_mhz']} MHz"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_max_ms / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": med_ms,
+        "ms_per_step_mean": sum(step_ms) / len(step_ms), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16x3" if precision == Bd.MH3A_BF16X3 else "f32",
         "data": "synthetic",
         "config": {"workload": f"decode B={B} N={N} (10 s stereo, 2 x 320000 samples) per GPU",
                    "global_batch": B * world, "latent_frames": N, "replicas": world,
-                   "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)"},
+                   "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)",
+                   "statistic": "median step"},
         "roofline": roofline,
         "roofline_activation": roofline_act,
         "e2e": {"value": e2e_value, "unit": UNIT,
@@ -372,11 +420,16 @@ def run_ours(args):
         "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16x3_tflops": p_tc, "fp32_tflops": p_fp32,
                   "source": peaks["source"]},
     }
+    if rank == 0 and world == 1 and not args.no_extra:
+        line["amp_stage"] = extra_amp_stage(Bd, PM, peaks, p_tc, p_fp32, flush, stream, dev,
+                                            max(args.steps, 10))
+    dec.close()
+    if rank == 0 and world == 1 and not args.no_extra:
+        line["batched_decode"] = extra_batched(S.workload_inputs(4), Bd, flush, stream, dev, 5)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_sample_frames)
+        line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    dec.close()
     if world > 1:
         dist.destroy_process_group()
 

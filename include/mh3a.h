@@ -53,8 +53,11 @@ typedef enum {
  *   MH3A_BF16X3   tensor cores (tcgen05): each fp32 operand is split into a bf16 head and a
  *                 bf16 tail, and the product is formed as head*head + head*tail + tail*head
  *                 with fp32 accumulation in tensor memory (about 16 significant bits per
- *                 operand).  Stages whose convolutions are too narrow for the tensor cores
- *                 run the fp32 CUDA-core kernels. */
+ *                 operand).  In this mode every convolution of the default architecture runs
+ *                 on the tensor cores -- conv_pre, the seven upsamplers and the AMP convs of
+ *                 all seven stages, 512 down to 8 channels -- and mh3a_decode and
+ *                 mh3a_amp_stage launch the same kernels for a stage.  Only the 1x1 input
+ *                 projection and the 8 -> 1 output conv are fp32 CUDA-core arithmetic. */
 typedef enum { MH3A_FP32 = 0, MH3A_BF16X3 = 1 } mh3a_precision;
 
 #define MH3A_FLAG_NO_CLAMP 1u /* return the waveform before the final clamp (testing)   */

@@ -59,7 +59,9 @@ def test_static_scratch_stage_matches_workspace_stage(precision):
     small = Bd.Decoder(arch, w, precision=precision, max_batch=1, max_frames=1)
     stream = torch.cuda.current_stream().cuda_stream
     try:
-        for stage, B, L in [(0, 2, 150), (3, 2, 3001), (5, 2, 9001)]:
+        # every stage width: several time tiles plus a ragged tail
+        for stage, B, L in [(0, 2, 150), (1, 2, 503), (2, 1, 2999), (3, 2, 3001), (4, 1, 10007),
+                            (5, 2, 9001), (6, 1, 40003)]:
             C_ = arch.stage_channels(stage)
             for call in range(2):
                 x = torch.from_numpy(S.make_stage_input(B, C_, L, 900 + 10 * stage + call)).to(dev)
@@ -68,6 +70,9 @@ def test_static_scratch_stage_matches_workspace_stage(precision):
                 st = f(small.handle, x.data_ptr(), B, L, stage, out.data_ptr(), stream)
                 assert st == 0, Bd.load().mh3a_last_error().decode()
                 torch.cuda.synchronize()
+                # a bounded pipeline wait that gave up would leave stale scratch behind
+                small.check_device_error()
+                ref_dec.check_device_error()
                 _close(out, ref, precision, f"stage {stage} call {call}")
         # beyond the static limit: rejected on the host with a clear message, output untouched
         C0 = arch.stage_channels(0)
