@@ -1,0 +1,686 @@
+// amp_fused.cu -- the narrow AMP stages (8 and 16 channels) as ONE kernel per stage: every CTA
+// runs a whole residual block over a window of time rows, all six layers of it, and keeps every
+// intermediate on chip.
+//
+// A residual block (FastVideo "minimax_h3_audio_vae" page, the `_amp_block` calls of
+// `MLXMiniMaxH3AudioVAE.decode`; the block body is the AMP1 reading: for each dilation d,
+// x <- x + conv_k,1(act(conv_k,d(act(x))))) is six layers.  At 8 and 16 channels each layer
+// is a thin contraction (K = 8..16 input channels per tap) over a long sequence, so the
+// separate activation and GEMM kernels of the wide stages spend their time moving the layer
+// tensors through HBM; here they never leave the SM:
+//
+//   x (fp32)  lives in tensor memory, one column per channel, lane = window row;
+//   v (fp32)  the activation's input, [channel][row] in shared memory, time-contiguous so that
+//             a lane's run of RUN rows is three 16-byte loads;
+//   A (bf16)  the activation written as the conv's 3xBF16 operand, heads and tails, rows of
+//             8 channels (the no-swizzle K-major core-matrix layout), in shared memory;
+//   D (fp32)  the conv's accumulators in tensor memory.
+//
+// Per layer:  act  v -> A  (CUDA cores; in place through v, then a transposing split)
+//             MMA  A x W -> D  (one thread; 2 tcgen05 MMAs per K-step, per 128-row tile)
+//             epi  D + bias -> v (conv_d) ;  x + D + bias -> x and v (conv_1)
+// The window is 1152 rows (9 tiles of 128); the block's receptive field (halo H rows per side:
+// per dilation 5 + d(k-1)/2 + 5 + (k-1)/2) is recomputed by neighbouring windows, and a CTA
+// writes its middle 1152 - 2H rows.  Rows outside the sequence follow the decode's padding:
+// the activation replicates the end samples (and its 2x-rate end values), the conv sees zeros.
+//
+// Precision: the same 3xBF16 products as the persistent GEMM; each accumulator receives one
+// layer's K-steps (at most 2 x 11 MMAs) and is folded into fp32 registers with round to nearest.
+//
+// Every mbarrier wait is bounded (1 s); a timeout sets the error flag and the CTA skips the rest
+// of its work with all barriers still reached, waits for its copies and MMAs, and returns.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "act_math.cuh"
+#include "tc_kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace mh3a {
+namespace {
+
+constexpr uint64_t kFwWait = 1000000000ull;   // ns
+constexpr int FW_MT = 9;                      // 128-row tiles per window
+constexpr int FW_WR = 128 * FW_MT;            // window rows
+constexpr int FW_RUN = 12;                    // activation outputs per lane
+constexpr int FW_WRUN = 32 * FW_RUN;          // rows per warp run (FW_WR = 3 runs)
+constexpr int FW_VM = 8;                      // margin rows of v on each side
+constexpr int FW_VS = FW_WR + 2 * FW_VM;      // floats per channel row of v
+constexpr int FW_PADO = 32;                   // margin rows of A on each side
+constexpr int FW_WO = FW_WR + 2 * FW_PADO;    // rows per channel group of A
+constexpr int FW_LAYERS = 2 * MH3A_MAX_DILATIONS;
+static_assert(FW_WR % FW_WRUN == 0, "whole warp runs per window");
+static_assert((FW_RUN * 4) % 16 == 0 && (FW_VS % 4) == 0, "16-byte aligned lane runs");
+
+// Per channel width: K-step layout of the weights and the tensor-memory columns.
+//   C = 8: a K-step is a tap pair (2 core columns = taps 2s, 2s+1 of 8 channels); its weight
+//          block holds per core column 24 rows [0 (8) | head (8) | tail (8)], so that
+//          MMA 1 = A_h [B_h | B_l] (rows 8..23) and MMA 2 = A_l [0 | B_h] (rows 0..15), both
+//          N = 16, land head x head in columns 0..7 and both cross products in 8..15.
+//   C = 16: a K-step is one tap (core columns = channel groups 0, 1); per core column 32 rows
+//          [head (16) | tail (16)]; MMA 1 = A_h [B_h | B_l] (N = 32), MMA 2 = A_l B_h (N = 16)
+//          into columns 16..31.
+template <int C>
+struct Fw {
+    static constexpr int G = C / 8;
+    static constexpr int BROWS = (C == 8) ? 24 : 32;              // weight rows per core column
+    static constexpr int KSB = 2 * BROWS * 16;                     // bytes per K-step block
+    static constexpr int MAXKS = (C == 8) ? 8 : 15;               // K <= 15
+    static constexpr int WBUF = MAXKS * KSB;
+    static constexpr int ACC = (C == 8) ? 16 : 32;                 // accumulator columns per tile
+    static constexpr int XCOL0 = FW_MT * ACC;                      // first column of x
+    static constexpr int USED = XCOL0 + FW_MT * C;
+    static constexpr int TCOLS = USED <= 32 ? 32 : USED <= 64 ? 64 : USED <= 128 ? 128 : USED <= 256 ? 256 : 512;
+    static constexpr int NCW = (C == 8) ? 8 : 16;                  // compute warps
+    static constexpr int NTHR = 64 + 32 * NCW;
+    static constexpr int OFF_A = C * FW_VS * 4;                    // v first
+    static constexpr int OFF_AL = OFF_A + G * FW_WO * 16;
+    static constexpr int OFF_W = OFF_AL + G * FW_WO * 16;
+    static constexpr int OFF_BAR = OFF_W + 2 * WBUF;
+    static constexpr int OFF_SEAM = OFF_BAR + 256;                // [NCW][8] floats
+    static constexpr int SMEM = OFF_SEAM + NCW * 8 * 4;
+    static_assert(USED <= 512, "tensor memory");
+    static_assert((OFF_A % 16) == 0 && (OFF_W % 128) == 0 && (OFF_BAR % 16) == 0, "alignment");
+};
+
+struct FwJob {
+    const uint16_t* w[FW_LAYERS];   // weight blob of each layer (K-step blocks)
+    const float* bias[FW_LAYERS];
+    const float* alpha[FW_LAYERS];  // SnakeBeta of the activation in front of each layer
+    const float* inv_beta[FW_LAYERS];
+    float* out;                     // [B, C, L] the block's output
+    int K;                          // kernel size
+    int dil[FW_LAYERS];             // dilation of each layer (1 for the second conv of a pair)
+    int H;                          // halo rows per side
+    int T;                          // output rows per window (FW_WR - 2 H)
+    int tiles;                      // windows per batch item
+    int unit0;                      // first CTA of the job
+};
+
+struct FwParams {
+    FwJob job[MH3A_MAX_RESBLOCKS];
+    int njobs, nlayers;
+    const float* x;                 // stage input [B, C, L]
+    int L, B;
+    ActFilter filt;
+    int* err;
+};
+
+__device__ __forceinline__ void cw_sync(int ncw) { asm volatile("bar.sync 1, %0;" ::"r"(ncw * 32) : "memory"); }
+
+// Two MMAs of one 3xBF16 K-step by one elected lane: D1 (+)= A1 B1 (idesc1), then D2 += A2 B2.
+__device__ __forceinline__ void mma_pair_elect(uint32_t d1, uint64_t a1, uint64_t b1, uint32_t idesc1, uint32_t d2,
+                                               uint64_t a2, uint64_t b2, uint32_t idesc2, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, q;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %8, 0;\n\t"
+        "setp.eq.b32 q, %8, %8;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%4], %5, %6, %7, q;\n\t}" ::"r"(d1),
+        "l"(a1), "l"(b1), "r"(idesc1), "r"(d2), "l"(a2), "l"(b2), "r"(idesc2), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                 "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// The C columns of x for one thread's row (32x32b: lane = row).
+template <int C>
+__device__ __forceinline__ void x_ld(uint32_t taddr, float (&v)[C]) {
+    if constexpr (C == 8) ptx::tmem_ld8(taddr, v);
+    else ptx::tmem_ld16(taddr, v);
+}
+template <int C>
+__device__ __forceinline__ void x_st(uint32_t taddr, const float (&v)[C]) {
+    if constexpr (C == 8) tmem_st8(taddr, v);
+    else tmem_st16(taddr, v);
+}
+
+// SnakeBeta value of 2x-rate index n (local: window rows x 2) from its six inputs q[k] =
+// v[base - k], base = floor(n / 2) + 2 + (n & 1): even n takes the odd taps of the
+// upsampler, odd n the even taps.
+__device__ __forceinline__ float snake_from6(const ActFilter& f, const float (&q)[6], int n, float al, float ib) {
+    const int par = (n & 1) ? 0 : 1;
+    float u = 0.f;
+#pragma unroll
+    for (int k = 0; k < 6; ++k) u = fmaf(par ? f.up[2 * k + 1] : f.up[2 * k], q[k], u);
+    return fmaf(actm::sin_sq_fast(al, u), ib, u);
+}
+
+// One warp run: rows [rw, rw + FW_WRUN) of one channel row `vr` (logical row 0 at vr[0];
+// margins of FW_VM rows on each side).  Lane l owns rows rs = rw + RUN l + [0, RUN).  The run's
+// inputs are taken into registers (act_load) before its outputs are written back over the
+// same rows (act_compute).  A warp runs the three runs of its channel in order, so the only
+// rows one run reads after another has overwritten them are the 8 rows left of its start:
+// those come from `seam`, where the warp stashed them before overwriting.
+struct ActIn {
+    float xv[FW_RUN + 12];   // v[rs - 8 + k]
+    float hq[6];             // halo lanes 0..9: the six inputs of their extra SnakeBeta value
+};
+
+__device__ __forceinline__ int halo_n(int lane, int rw) {
+    // lanes 0..4: the five 2x-rate values left of lane 0's run; 5..9: right of lane 31's run
+    return lane < 5 ? 2 * rw - 5 + lane : 2 * (rw + FW_WRUN) + (lane - 5);
+}
+
+// seam: the 8 input rows [rw - 8, rw), or null when they are still intact in vr.
+__device__ __forceinline__ void act_load(const float* vr, const float* seam, int rw, ActIn& in) {
+    const int lane = threadIdx.x & 31;
+    const int rs = rw + FW_RUN * lane;
+#pragma unroll
+    for (int k = 0; k < (FW_RUN + 12) / 4; ++k) {
+        const float4 q = (seam && lane == 0 && k < 2) ? *reinterpret_cast<const float4*>(seam + 4 * k)
+                                                      : *reinterpret_cast<const float4*>(vr + rs - 8 + 4 * k);
+        in.xv[4 * k] = q.x;
+        in.xv[4 * k + 1] = q.y;
+        in.xv[4 * k + 2] = q.z;
+        in.xv[4 * k + 3] = q.w;
+    }
+    if (lane < 10) {
+        const int n = halo_n(lane, rw);
+        const int base = (n >> 1) + 2 + (n & 1);
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int r = base - k;
+            in.hq[k] = (seam && r < rw) ? seam[r - rw + 8] : vr[r];
+        }
+    }
+}
+
+// rw: first window row of the run; tw: sequence time of window row 0; L: sequence length.
+template <bool EDGE>
+__device__ __forceinline__ void act_compute(const ActFilter& f, const ActIn& in, float al, float ib, int rw, int tw,
+                                            int L, float (&a)[FW_RUN]) {
+    constexpr int RUN = FW_RUN;
+    constexpr int NS = 2 * RUN + 10;
+    const int lane = threadIdx.x & 31;
+    const int rs = rw + RUN * lane;
+    float s[NS];
+    // own values: s[5 + i] at local 2x index 2 rs + i
+#pragma unroll
+    for (int i = 0; i < 2 * RUN; ++i) {
+        float u = 0.f;
+        if (i % 2 == 0) {
+#pragma unroll
+            for (int q = 0; q < 6; ++q) u = fmaf(f.up[2 * q + 1], in.xv[i / 2 + 10 - q], u);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 6; ++q) u = fmaf(f.up[2 * q], in.xv[(i - 1) / 2 + 11 - q], u);
+        }
+        s[5 + i] = fmaf(actm::sin_sq_fast(al, u), ib, u);
+    }
+    float hv = 0.f;
+    if (lane < 10) hv = snake_from6(f, in.hq, halo_n(lane, rw), al, ib);
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+        const float from_left = __shfl_up_sync(0xffffffffu, s[j + 2 * RUN], 1);
+        const float from_right = __shfl_down_sync(0xffffffffu, s[j + 5], 1);
+        const float h = __shfl_sync(0xffffffffu, hv, (lane == 31) ? j + 5 : j);
+        s[j] = (lane == 0) ? h : from_left;
+        s[j + 5 + 2 * RUN] = (lane == 31) ? h : from_right;
+    }
+    if (EDGE) {
+        // the 2x-rate signal is replicate-padded: true index n < 0 takes s(0), n > 2L - 1 takes
+        // s(2L - 1); s[j] sits at true index 2 (tw + rs) - 5 + j
+        const int n0 = 2 * (tw + rs) - 5;
+        const int j0 = -n0, je = 2 * L - 1 - n0;
+        float sf = s[0], sl = s[NS - 1];
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            sf = (j == j0) ? s[j] : sf;
+            sl = (j == je) ? s[j] : sl;
+        }
+#pragma unroll
+        for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
+    }
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(f.down[j], s[2 * i + j], v);
+        a[i] = v;
+    }
+}
+
+template <int C>
+__global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(const FwParams p) {
+    using F = Fw<C>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    ptx::grid_dep_wait();   // launched as a programmatic dependent (see launch_dependent)
+    float* vbuf = reinterpret_cast<float*>(smem);                      // [C][FW_VS]
+    uint8_t* a_hi = smem + F::OFF_A;                                   // [G][FW_WO][16 B]
+    uint8_t* a_lo = smem + F::OFF_AL;
+    uint8_t* wbuf = smem + F::OFF_W;                                   // [2][WBUF]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
+    uint64_t* w_full = bars;          // [2]
+    uint64_t* w_empty = bars + 2;     // [2]
+    uint64_t* op_full = bars + 4;     // A operand of the current layer written
+    uint64_t* done_bar = bars + 5;    // every MMA issued has completed
+    uint64_t* acc_full = bars + 6;    // [FW_MT] per tile: the layer's MMAs of the tile completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + FW_MT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the unit of this CTA: job (heaviest first), batch item, window
+    int z = 0;
+    while (z + 1 < p.njobs && (int)blockIdx.x >= p.job[z + 1].unit0) ++z;
+    const FwJob& J = p.job[z];
+    const int u = blockIdx.x - J.unit0;
+    const int b = u / J.tiles, tile = u - b * J.tiles;
+    const int L = p.L;
+    const int t0 = tile * J.T;            // first output row (sequence time)
+    const int tw = t0 - J.H;              // sequence time of window row 0
+    const int r_lo = max(0, -tw), r_hi = min(FW_WR, L - tw);   // window rows inside the sequence
+    const int nl = p.nlayers;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&w_full[i], 1);
+            ptx::mbar_init(&w_empty[i], 1);
+        }
+        ptx::mbar_init(op_full, 1);
+        ptx::mbar_init(done_bar, 1);
+        for (int i = 0; i < FW_MT; ++i) ptx::mbar_init(&acc_full[i], 1);
+        *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, F::TCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc1 = ptx::idesc_bf16(128, C == 8 ? 16 : 32);
+        constexpr uint32_t idesc2 = ptx::idesc_bf16(128, 16);
+        constexpr uint32_t b_lbo = F::BROWS * 16;
+        const uint32_t ahs = ptx::smem_u32(a_hi), als = ptx::smem_u32(a_lo), ws = ptx::smem_u32(wbuf);
+        bool ok = *abort_flag == 0;
+        for (int l = 0; l < nl && ok; ++l) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(op_full, l & 1, kFwWait));
+            if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&w_full[l & 1], (l >> 1) & 1, kFwWait));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const int d = J.dil[l];
+            const int pad = d * (J.K - 1) / 2;
+            const int KS = (C == 8) ? (J.K + 1) / 2 : J.K;
+            const uint32_t a_lbo = (C == 8) ? (uint32_t)d * 16u : (uint32_t)FW_WO * 16u;
+            const uint32_t wb = ws + (uint32_t)((l & 1) * F::WBUF);
+            for (int i = 0; i < FW_MT; ++i) {
+                const uint32_t dcol = tmem + (uint32_t)(i * F::ACC);
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int row = 128 * i + ((C == 8) ? 2 * ks : ks) * d - pad + FW_PADO;
+                    const uint64_t ah = ptx::desc64(ptx::desc_lo(ahs + (uint32_t)row * 16u, a_lbo));
+                    const uint64_t al = ptx::desc64(ptx::desc_lo(als + (uint32_t)row * 16u, a_lbo));
+                    const uint32_t bb = wb + (uint32_t)(ks * F::KSB);
+                    if constexpr (C == 8) {
+                        const uint64_t b1 = ptx::desc64(ptx::desc_lo(bb + 128u, b_lbo));   // [B_h | B_l]
+                        const uint64_t b2 = ptx::desc64(ptx::desc_lo(bb, b_lbo));          // [0 | B_h]
+                        mma_pair_elect(dcol, ah, b1, idesc1, dcol, al, b2, idesc2, ks > 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t b1 = ptx::desc64(ptx::desc_lo(bb, b_lbo));
+                        mma_pair_elect(dcol, ah, b1, idesc1, dcol + 16u, al, b1, idesc2, ks > 0 ? 1u : 0u);
+                    }
+                }
+                ptx::mma_commit_elect(&acc_full[i]);
+            }
+            ptx::mma_commit_elect(&w_empty[l & 1]);
+            if (*abort_flag) ok = false;
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(p.err, 11);
+        }
+        // every MMA issued has completed before tensor memory is released
+        ptx::mma_commit_elect(done_bar);
+        ptx::mbar_wait(done_bar, 0, kFwWait);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ weight loader
+        if (lane == 0) {
+            bool ok = *abort_flag == 0;
+            int issued = 0;
+            for (int l = 0; l < nl && ok; ++l) {
+                const int KS = (C == 8) ? (J.K + 1) / 2 : J.K;
+                const uint32_t bytes = (uint32_t)(KS * F::KSB);
+                if (!ptx::mbar_wait(&w_empty[l & 1], ((l >> 1) & 1) ^ 1, kFwWait) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&w_full[l & 1], bytes);
+                ptx::bulk_g2s(wbuf + (l & 1) * F::WBUF, J.w[l], bytes, &w_full[l & 1]);
+                issued = l + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(p.err, 12);
+            }
+            // the copies in flight land before the CTA may exit
+            for (int l = (issued > 2 ? issued - 2 : 0); l < issued; ++l)
+                ptx::mbar_wait(&w_full[l & 1], (l >> 1) & 1, kFwWait);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ compute warps
+        constexpr int NCW = F::NCW;
+        const int cw = warp - 2;
+        const int ct = threadIdx.x - 64;
+        const int q4 = warp & 3;                   // tensor-memory lane quarter of this warp
+        const int sub = cw >> 2, nsub = NCW / 4;   // this warp's share of the tiles
+        bool ok = *abort_flag == 0;
+        // zero the operand margins once (read only by rows that are never written out)
+        for (int i = ct; i < 2 * F::G * FW_WO; i += NCW * 32) {
+            uint8_t* base = (i < F::G * FW_WO) ? a_hi : a_lo;
+            const int k = i % (F::G * FW_WO);
+            *reinterpret_cast<uint4*>(base + (size_t)k * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        // the input window (replicate padding: the time index is clamped into the sequence)
+        {
+            const float* xb = p.x + (long long)b * C * L;
+            for (int i = ct; i < C * FW_VS; i += NCW * 32) {
+                const int c = i / FW_VS, r = i - c * FW_VS - FW_VM;
+                const int t = min(max(tw + r, 0), L - 1);
+                ptx::cp_async4(vbuf + i, xb + (long long)c * L + t);
+            }
+            ptx::cp_async_commit();
+            ptx::cp_async_wait_all();
+        }
+        cw_sync(NCW);
+        // x into tensor memory
+        for (int i = sub; i < FW_MT; i += nsub) {
+            const int r = 128 * i + 32 * q4 + lane;
+            float xv[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) xv[c] = vbuf[c * FW_VS + FW_VM + r];
+            x_st<C>(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(F::XCOL0 + i * C), xv);
+        }
+        tmem_wait_st();
+        const bool edge = r_lo > 0 || r_hi < FW_WR;
+        for (int l = 0; l < nl; ++l) {
+            // ---- activation of v into the A operand
+            if (edge) {
+                // replicate padding of the activation's input: rows outside the sequence take
+                // the end samples (their current contents are not the signal there)
+                for (int i = ct; i < C * FW_VS; i += NCW * 32) {
+                    const int c = i / FW_VS, r = i - c * FW_VS - FW_VM;
+                    if (r < r_lo) vbuf[i] = vbuf[c * FW_VS + FW_VM + r_lo];
+                    else if (r >= r_hi) vbuf[i] = vbuf[c * FW_VS + FW_VM + r_hi - 1];
+                }
+                cw_sync(NCW);
+            }
+            // one channel per warp, its runs in order (see act_load)
+            static_assert(F::NCW == C, "one compute warp per channel");
+            {
+                const int c = cw;
+                float* vr = vbuf + c * FW_VS + FW_VM;
+                float* seam = reinterpret_cast<float*>(smem + F::OFF_SEAM) + cw * 8;
+                const float al = __ldg(J.alpha[l] + c), ib = __ldg(J.inv_beta[l] + c);
+#pragma unroll 1
+                for (int k = 0; k < FW_WR / FW_WRUN; ++k) {
+                    const int rw = k * FW_WRUN;
+                    ActIn in;
+                    act_load(vr, k > 0 ? seam : nullptr, rw, in);
+                    __syncwarp();
+                    // the next run's left input rows, before this run overwrites them
+                    if (k + 1 < FW_WR / FW_WRUN && lane < 8) seam[lane] = vr[rw + FW_WRUN - 8 + lane];
+                    __syncwarp();
+                    if (ok) {
+                        float a[FW_RUN];
+                        // the run's 2x-rate window reaches past a sequence end
+                        const bool e = (tw + rw - 8 < 0) || (tw + rw + FW_WRUN + 8 > L);
+                        if (e) act_compute<true>(p.filt, in, al, ib, rw, tw, L, a);
+                        else act_compute<false>(p.filt, in, al, ib, rw, tw, L, a);
+                        float* dst = vr + rw + FW_RUN * lane;
+#pragma unroll
+                        for (int q = 0; q < FW_RUN / 4; ++q)
+                            *reinterpret_cast<float4*>(dst + 4 * q) =
+                                make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                    }
+                    __syncwarp();
+                }
+            }
+            cw_sync(NCW);
+            // transposing split: rows of 8 channels, heads and tails; zeros outside the sequence
+            if (ok) {
+                for (int i = ct; i < F::G * FW_WR; i += NCW * 32) {
+                    const int g = i / FW_WR, r = i - g * FW_WR;
+                    float v[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) v[c] = vbuf[(8 * g + c) * FW_VS + FW_VM + r];
+                    uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;
+                    if (r >= r_lo && r < r_hi) {
+                        actm::split2(v[0], v[1], &hv.x, &lv.x);
+                        actm::split2(v[2], v[3], &hv.y, &lv.y);
+                        actm::split2(v[4], v[5], &hv.z, &lv.z);
+                        actm::split2(v[6], v[7], &hv.w, &lv.w);
+                    }
+                    const size_t off = ((size_t)g * FW_WO + FW_PADO + r) * 16;
+                    *reinterpret_cast<uint4*>(a_hi + off) = hv;
+                    *reinterpret_cast<uint4*>(a_lo + off) = lv;
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            cw_sync(NCW);
+            if (ct == 0) ptx::mbar_arrive(op_full);
+            // ---- epilogue of the layer's conv, tile by tile as the MMAs complete
+            const bool second = (l & 1) != 0;
+            float bias[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) bias[c] = __ldg(J.bias[l] + c);
+            for (int i = sub; i < FW_MT; i += nsub) {
+                if (ok && *abort_flag) ok = false;
+                if (ok && !ptx::mbar_wait(&acc_full[i], l & 1, kFwWait)) {
+                    ok = false;
+                    *abort_flag = 1;
+                    atomicExch(p.err, 13);
+                }
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    continue;
+                }
+                ptx::tc_fence_after();
+                const int r = 128 * i + 32 * q4 + lane;
+                const uint32_t lq = (uint32_t)(32 * q4) << 16;
+                float y[C];
+                if constexpr (C == 8) {
+                    float v[16];
+                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) y[c] = (v[c] + v[8 + c]) + bias[c];
+                } else {
+                    float v0[16], v1[16];
+                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v0);
+                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC + 16), v1);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) y[c] = (v0[c] + v1[c]) + bias[c];
+                }
+                if (second) {
+                    float xo[C];
+                    const uint32_t xa = tmem + lq + (uint32_t)(F::XCOL0 + i * C);
+                    x_ld<C>(xa, xo);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) y[c] = xo[c] + y[c];
+                    if (l + 1 < nl) x_st<C>(xa, y);
+                }
+#pragma unroll
+                for (int c = 0; c < C; ++c) vbuf[c * FW_VS + FW_VM + r] = y[c];
+            }
+            tmem_wait_st();
+            ptx::tc_fence_before();
+            cw_sync(NCW);
+        }
+        // ---- the window's output rows
+        if (ok) {
+            const int n_out = min(J.T, L - t0);
+            float* ob = J.out + (long long)b * C * L + t0;
+            for (int i = ct; i < C * n_out; i += NCW * 32) {
+                const int c = i / n_out, k = i - c * n_out;
+                ob[(long long)c * L + k] = vbuf[c * FW_VS + FW_VM + J.H + k];
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            atomicExch(p.err, 14);
+        }
+    }
+    ptx::grid_dep_launch();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 0) ptx::tmem_dealloc(tmem, F::TCOLS);
+}
+
+template <int C>
+int launch_fused(const FwParams& p, int units, cudaStream_t s) {
+    using F = Fw<C>;
+    auto kern = k_amp_fused<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM) != cudaSuccess) return -1;
+    return launch_dependent(kern, dim3(units), dim3(F::NTHR), F::SMEM, s, p) == cudaSuccess ? 1 : -1;
+}
+
+uint16_t bf16_rn_bits(float v) {
+    uint32_t u;
+    std::memcpy(&u, &v, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+float bf16_bits_value(uint16_t h) {
+    const uint32_t u = (uint32_t)h << 16;
+    float v;
+    std::memcpy(&v, &u, 4);
+    return v;
+}
+
+}  // namespace
+
+int fused_halo(int K, const int* dil, int nd) {
+    int H = 0;
+    for (int m = 0; m < nd; ++m) H += 5 + dil[m] * (K - 1) / 2 + 5 + (K - 1) / 2;
+    return H;
+}
+
+bool fused_stage_supported(int C, const mh3a_config& c) {
+    // 16 channels measured slower fused (one CTA per SM) than as separate activation and GEMM
+    // launches; the 16-channel instantiation is kept for that comparison.
+    if (C != 8) return false;
+    if (c.n_resblocks < 1 || c.n_resblocks > MH3A_MAX_RESBLOCKS || c.n_dilations < 1) return false;
+    for (int j = 0; j < c.n_resblocks; ++j) {
+        const int K = c.rb_kernels[j];
+        if (K > 15 || K % 2 == 0) return false;
+        for (int m = 0; m < c.n_dilations; ++m) {
+            const int d = c.rb_dilations[j][m];
+            // rows an MMA reads stay inside the operand's margins
+            const int reach = (C == 8) ? (2 * ((K + 1) / 2) - 1) * d - d * (K - 1) / 2 : d * (K - 1) / 2;
+            if (d * (K - 1) / 2 > FW_PADO || reach > FW_PADO) return false;
+        }
+        // at least one 128-row tile of output per window
+        if (FW_WR - 2 * fused_halo(K, c.rb_dilations[j], c.n_dilations) < 128) return false;
+    }
+    return true;
+}
+
+// Weight blob of one layer: [K-step][core column][row][8 bf16] (see Fw).
+void prepare_fused_conv(const std::vector<float>& w_oik, int C, int K, TcConv* out) {
+    const int KS = (C == 8) ? (K + 1) / 2 : K;
+    const int BROWS = (C == 8) ? 24 : 32;
+    std::vector<uint16_t> buf((size_t)KS * 2 * BROWS * 8, 0);
+    size_t pos = 0;
+    for (int ks = 0; ks < KS; ++ks)
+        for (int cc = 0; cc < 2; ++cc)
+            for (int n = 0; n < BROWS; ++n)
+                for (int e = 0; e < 8; ++e, ++pos) {
+                    int o = -1, part = 0;
+                    if (C == 8) {
+                        if (n >= 8) { o = (n - 8) % 8; part = (n >= 16) ? 1 : 0; }
+                    } else {
+                        o = n % 16;
+                        part = (n >= 16) ? 1 : 0;
+                    }
+                    const int tap = (C == 8) ? 2 * ks + cc : ks;
+                    const int ci = (C == 8) ? e : 8 * cc + e;
+                    if (o < 0 || tap >= K) continue;
+                    const float v = w_oik[((size_t)o * C + ci) * K + tap];
+                    const uint16_t hb = bf16_rn_bits(v);
+                    buf[pos] = part == 0 ? hb : bf16_rn_bits(v - bf16_bits_value(hb));
+                }
+    out->staging.assign((buf.size() + 1) / 2, 0.f);
+    std::memcpy(out->staging.data(), buf.data(), buf.size() * sizeof(uint16_t));
+    out->cout = C;
+    out->cin = C;
+    out->k = K;
+}
+
+int launch_amp_fused(const ConvParams* layers, int nlayers, int njobs, const TcStageWeights& w, const float* x,
+                     cudaStream_t s, int* err) {
+    const int C = layers[0].Cin;
+    if (nlayers > FW_LAYERS || nlayers % 2 != 0 || njobs > MH3A_MAX_RESBLOCKS) return -1;
+    FwParams p{};
+    p.njobs = njobs;
+    p.nlayers = nlayers;
+    p.x = x;
+    p.L = layers[0].L;
+    p.B = layers[0].B;
+    p.filt = layers[0].filt;
+    p.err = err;
+    // heaviest job first: the largest halo (and kernel) starts earliest
+    int order[MH3A_MAX_RESBLOCKS];
+    for (int j = 0; j < njobs; ++j) order[j] = j;
+    std::sort(order, order + njobs, [&](int a, int b) { return layers[0].job[a].K > layers[0].job[b].K; });
+    int units = 0;
+    for (int z = 0; z < njobs; ++z) {
+        const int j = order[z];
+        FwJob& J = p.job[z];
+        J.K = layers[0].job[j].K;
+        int dil[MH3A_MAX_DILATIONS];
+        for (int l = 0; l < nlayers; ++l) {
+            const ConvJob& cj = layers[l].job[j];
+            const TcConv& tw = w.conv[j][l / 2][l % 2];
+            if (!tw.dev || cj.K != J.K) return -1;
+            J.w[l] = reinterpret_cast<const uint16_t*>(tw.dev);
+            J.bias[l] = cj.bias;
+            J.alpha[l] = cj.alpha;
+            J.inv_beta[l] = cj.inv_beta;
+            J.dil[l] = cj.dil;
+            if (l % 2 == 0) dil[l / 2] = cj.dil;
+        }
+        J.out = layers[nlayers - 1].job[j].out;
+        J.H = fused_halo(J.K, dil, nlayers / 2);
+        J.T = FW_WR - 2 * J.H;
+        if (J.T < 128) return -1;
+        J.tiles = (p.L + J.T - 1) / J.T;
+        J.unit0 = units;
+        units += p.B * J.tiles;
+    }
+    if (C == 8) return launch_fused<8>(p, units, s);
+    if (C == 16) return launch_fused<16>(p, units, s);
+    return -1;
+}
+
+}  // namespace mh3a

@@ -112,8 +112,10 @@ struct mh3a_handle {
     DevAct act_post;
     TcStageWeights tc[MH3A_MAX_STAGES];   // tensor-core operand copies (BF16X3)
     bool stage_tc[MH3A_MAX_STAGES] = {};
+    bool stage_fused[MH3A_MAX_STAGES] = {};   // narrow stages: one fused kernel per stage
     bool pre_tc = false;                  // conv_pre on the tensor cores
     bool ups_tc[MH3A_MAX_STAGES] = {};    // transposed convs on the tensor cores
+    mh3a_allocator alloc{};               // caller's device allocator (alloc == NULL: cudaMalloc)
     char* warena = nullptr;
     size_t wbytes = 0;
     // workspace
@@ -143,6 +145,7 @@ struct mh3a_handle {
     cudaEvent_t kev[6][3] = {};
     bool kev_made = false;
     int kev_rec = -1;                       // the stage the last decode recorded
+    bool kev_fused = false;                 // it was a fused stage: one launch, kev[0][0..1]
     long long launches = 0;
 };
 
@@ -172,6 +175,33 @@ mh3a_status validate(const mh3a_config& c) {
     if (c.precision != MH3A_FP32 && c.precision != MH3A_BF16X3) return MH3A_ERR_CONFIG;
     if (c.max_batch < 1 || c.max_frames < 1) return MH3A_ERR_CONFIG;
     return MH3A_OK;
+}
+
+// Device memory of a handle: from the caller's allocator when one was given, else cudaMalloc.
+bool dev_alloc(mh3a_handle* h, size_t bytes, char** out) {
+    *out = nullptr;
+    if (h->alloc.alloc) {
+        void* p = h->alloc.alloc(bytes, h->alloc.user);
+        if (!p || (reinterpret_cast<uintptr_t>(p) & 255) != 0) {
+            if (p) h->alloc.release(p, h->alloc.user);   // misaligned: not usable
+            return false;
+        }
+        *out = static_cast<char*>(p);
+        return true;
+    }
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+        cudaGetLastError();   // the failed allocation is reported as MH3A_ERR_ALLOC, not left pending
+        return false;
+    }
+    *out = static_cast<char*>(p);
+    return true;
+}
+
+void dev_free(mh3a_handle* h, char* p) {
+    if (!p) return;
+    if (h->alloc.alloc) h->alloc.release(p, h->alloc.user);
+    else cudaFree(p);
 }
 
 // Host staging of the folded weights before one device copy.
@@ -296,6 +326,7 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
     const mh3a_config& c = h->cfg;
     const int C = stage_channels(c, stage);
     const int nrb = c.n_resblocks;
+    ConvParams layers[2 * MH3A_MAX_DILATIONS];
     for (int m = 0; m < c.n_dilations; ++m) {
         for (int half = 0; half < 2; ++half) {
             ConvParams p{};
@@ -321,6 +352,10 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                 J.K = k;
                 J.dil = d;
                 J.pad = d * (k - 1) / 2;
+            }
+            if (h->stage_fused[stage]) {
+                layers[2 * m + half] = p;   // launched below, all layers at once
+                continue;
             }
             int n;
             if (h->stage_tc[stage]) {
@@ -353,13 +388,27 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                 n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err, h->dev_err + 16);
                 if (kprof && n > 0) {
                     CK_CUDA(cudaEventRecord(h->kev[li][2], s), "cudaEventRecord");
-                    if (li == 5) h->kev_rec = stage;
+                    if (li == 5) {
+                        h->kev_rec = stage;
+                        h->kev_fused = false;
+                    }
                 }
             } else {
                 n = launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             }
             mh3a_status st = counted(h, n);
             if (st) return st;
+        }
+    }
+    if (h->stage_fused[stage]) {
+        const bool kprof = h->kprof_stage == stage && h->kev_made;
+        if (kprof) CK_CUDA(cudaEventRecord(h->kev[0][0], s), "cudaEventRecord");
+        mh3a_status st = counted(h, launch_amp_fused(layers, 2 * c.n_dilations, nrb, h->tc[stage], in, s, h->dev_err));
+        if (st) return st;
+        if (kprof) {
+            CK_CUDA(cudaEventRecord(h->kev[0][1], s), "cudaEventRecord");
+            h->kev_rec = stage;
+            h->kev_fused = true;
         }
     }
     return MH3A_OK;
@@ -680,19 +729,26 @@ void mh3a_destroy(mh3a_handle* h) {
     for (auto& li : h->kev)
         for (auto& e : li)
             if (e) cudaEventDestroy(e);
-    if (h->warena) cudaFree(h->warena);
-    if (h->arena) cudaFree(h->arena);
+    dev_free(h, h->warena);
+    dev_free(h, h->arena);
     cudaSetDevice(prev);
     delete h;
 }
 
 mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int n_weights, mh3a_handle** out) {
+    return mh3a_create_with_allocator(cfg, weights, n_weights, nullptr, out);
+}
+
+mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh3a_tensor* weights, int n_weights,
+                                       const mh3a_allocator* allocator, mh3a_handle** out) {
     if (out) *out = nullptr;
     if (!cfg || !weights || !out || n_weights < 1) return MH3A_ERR_INVALID_ARG;
+    if (allocator && (!allocator->alloc || !allocator->release)) return MH3A_ERR_INVALID_ARG;
     mh3a_status st = validate(*cfg);
     if (st) return st;
     mh3a_handle* h = new (std::nothrow) mh3a_handle();
     if (!h) return MH3A_ERR_ALLOC;
+    if (allocator) h->alloc = *allocator;
     h->cfg = *cfg;
     h->cfg.latents_mean = nullptr;  // folded below; the caller's arrays are not retained
     h->cfg.latents_std = nullptr;
@@ -759,6 +815,7 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
             return fail(st);
         if (h->ups_tc[i]) prepare_tc_convt(iok, C, Co, c.kernels[i], c.rates[i], &h->tc[i].ups);
         h->stage_tc[i] = (c.precision == MH3A_BF16X3) && tc_stage_supported(Co, c);
+        h->stage_fused[i] = h->stage_tc[i] && fused_stage_supported(Co, c);
         for (int j = 0; j < c.n_resblocks; ++j) {
             const int k = c.rb_kernels[j];
             const int rb = i * c.n_resblocks + j;
@@ -771,7 +828,10 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
                 std::snprintf(buf, sizeof buf, "decoder.resblocks.%d.convs2.%d", rb, m);
                 if ((st = fold_conv(lk, buf, Co, Co, k, true, ha, &h->rb2[i][j][m], tc ? &oik2 : nullptr)))
                     return fail(st);
-                if (tc) {
+                if (tc && h->stage_fused[i]) {
+                    prepare_fused_conv(oik1, Co, k, &h->tc[i].conv[j][m][0]);
+                    prepare_fused_conv(oik2, Co, k, &h->tc[i].conv[j][m][1]);
+                } else if (tc) {
                     prepare_tc_conv(oik1, Co, k, &h->tc[i].conv[j][m][0]);
                     prepare_tc_conv(oik2, Co, k, &h->tc[i].conv[j][m][1]);
                 }
@@ -793,13 +853,7 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
     // tensor-core operand copies go into the same arena
     for (int i = 0; i < c.n_stages; ++i) tc_register(&h->tc[i], [&](const std::vector<float>& v, float** d) { ha.add(v, d); });
 
-    // one device copy of every folded weight
     h->wbytes = ha.data.size() * sizeof(float);
-    if (cudaMalloc(&h->warena, h->wbytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
-    if (cudaMemcpy(h->warena, ha.data.data(), h->wbytes, cudaMemcpyHostToDevice) != cudaSuccess)
-        return fail(cuda_fail(cudaGetLastError(), "weight upload"));
-    for (auto& f : ha.fix) *f.dst = reinterpret_cast<float*>(h->warena) + f.off;
-    for (int i = 0; i < c.n_stages; ++i) tc_finalize(&h->tc[i]);
 
     // workspace: stage buffers sized for the widest stage at max_batch x max_frames
     long long cap = 0, len = 1;
@@ -827,14 +881,28 @@ mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int 
             if (h->ups_tc[i]) need = std::max(need, (long long)Cin * (Lin + pads));
             Lin *= c.rates[i];
             Cin /= 2;
-            if (h->stage_tc[i]) need = std::max(need, (long long)Cin * (Lin + pads));
+            if (h->stage_tc[i] && !h->stage_fused[i]) need = std::max(need, (long long)Cin * (Lin + pads));
         }
         h->a_cap = need * c.max_batch;
     }
     const long long n_a = rnd((h->a_cap + 1) / 2);   // floats per head or tail array
     const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64 + 2 * c.n_resblocks * n_a;
     h->abytes = (size_t)total * sizeof(float);
-    if (cudaMalloc(&h->arena, h->abytes) != cudaSuccess) return fail(MH3A_ERR_ALLOC);
+    // both device allocations before any device work, so that a failed one leaves nothing behind
+    // but what fail() releases
+    if (!dev_alloc(h, h->wbytes, &h->warena)) {
+        g_last_error = "device allocation of the weights failed";
+        return fail(MH3A_ERR_ALLOC);
+    }
+    if (!dev_alloc(h, h->abytes, &h->arena)) {
+        g_last_error = "device allocation of the workspace failed";
+        return fail(MH3A_ERR_ALLOC);
+    }
+    // one device copy of every folded weight
+    if (cudaMemcpy(h->warena, ha.data.data(), h->wbytes, cudaMemcpyHostToDevice) != cudaSuccess)
+        return fail(cuda_fail(cudaGetLastError(), "weight upload"));
+    for (auto& f : ha.fix) *f.dst = reinterpret_cast<float*>(h->warena) + f.off;
+    for (int i = 0; i < c.n_stages; ++i) tc_finalize(&h->tc[i]);
     float* p = reinterpret_cast<float*>(h->arena);
     h->buf_in = p; p += n_in;
     h->buf_pre = p; p += n_pre;
@@ -924,6 +992,12 @@ mh3a_status mh3a_stage_kernel_times(mh3a_handle* h, int stage, float* act_ms, fl
     *act_ms = 0.f;
     *gemm_ms = 0.f;
     if (!h->kev_made || h->kev_rec != stage) return MH3A_ERR_UNSUPPORTED;
+    if (h->kev_fused) {
+        // one fused launch does the whole stage: its time is reported as the GEMM time
+        CK_CUDA(cudaEventSynchronize(h->kev[0][1]), "cudaEventSynchronize");
+        CK_CUDA(cudaEventElapsedTime(gemm_ms, h->kev[0][0], h->kev[0][1]), "cudaEventElapsedTime");
+        return MH3A_OK;
+    }
     CK_CUDA(cudaEventSynchronize(h->kev[5][2]), "cudaEventSynchronize");
     for (int li = 0; li < 6; ++li) {
         float a = 0.f, g = 0.f;

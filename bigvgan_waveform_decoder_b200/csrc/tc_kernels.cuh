@@ -48,6 +48,18 @@ void tc_register(TcStageWeights* w, AddFn add) {
         if (!c.staging.empty()) add(c.staging, &c.dev);
 }
 
+// The narrow AMP stages (8 and 16 channels) as one fused kernel per stage (amp_fused.cu): each
+// CTA runs all layers of one residual block over a window of rows, intermediates on chip.
+bool fused_stage_supported(int C, const mh3a_config& c);
+// One layer's weights ([O, I, K] folded fp32) in the fused kernel's K-step layout.
+void prepare_fused_conv(const std::vector<float>& w_oik, int C, int K, TcConv* out);
+// `layers[l]` (l = 0 .. nlayers-1, two per dilation: the dilated conv, then the k x 1 conv)
+// describe the stage's layers for all `njobs` residual blocks as the per-layer launches would
+// (weights, biases, activations, dilations); the stage input is x and block j's output goes to
+// layers[nlayers-1].job[j].out.  Weights come from w.conv[j][l / 2][l % 2] (prepare_fused_conv).
+int launch_amp_fused(const ConvParams* layers, int nlayers, int njobs, const TcStageWeights& w, const float* x,
+                     cudaStream_t s, int* err);
+
 // Drop host staging once the device copy exists.
 void tc_finalize(TcStageWeights* w);
 
