@@ -22,7 +22,8 @@ MAX_STAGES, MAX_RESBLOCKS, MAX_DILATIONS = 8, 4, 4
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "shape mismatch",
           4: "missing weight", 5: "allocation failed", 6: "CUDA error", 7: "unsupported request"}
 
-EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_decode", "mh3a_decode_host",
+EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_create_with_allocator", "mh3a_decode",
+           "mh3a_decode_host",
            "mh3a_amp_stage", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
            "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error",
            "mh3a_stage_uses_tensor_cores", "mh3a_segment_uses_tensor_cores",
@@ -60,6 +61,14 @@ class mh3a_tensor(C.Structure):
     ]
 
 
+ALLOC_FN = C.CFUNCTYPE(C.c_void_p, C.c_size_t, C.c_void_p)
+RELEASE_FN = C.CFUNCTYPE(None, C.c_void_p, C.c_void_p)
+
+
+class mh3a_allocator(C.Structure):
+    _fields_ = [("alloc", ALLOC_FN), ("release", RELEASE_FN), ("user", C.c_void_p)]
+
+
 class MH3AError(RuntimeError):
     def __init__(self, status: int, what: str, detail: str = ""):
         self.status = status
@@ -86,6 +95,9 @@ def load():
     L.mh3a_default_config.restype = None
     L.mh3a_create.argtypes = [C.POINTER(mh3a_config), C.POINTER(mh3a_tensor), C.c_int, C.POINTER(vp)]
     L.mh3a_create.restype = C.c_int
+    L.mh3a_create_with_allocator.argtypes = [C.POINTER(mh3a_config), C.POINTER(mh3a_tensor), C.c_int,
+                                             C.POINTER(mh3a_allocator), C.POINTER(vp)]
+    L.mh3a_create_with_allocator.restype = C.c_int
     L.mh3a_decode.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
     L.mh3a_decode.restype = C.c_int
     L.mh3a_decode_host.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
@@ -188,7 +200,10 @@ class Decoder:
     """Owns one mh3a handle on the current CUDA device."""
 
     def __init__(self, arch, weights: dict, precision: int = MH3A_BF16X3, max_batch: int = 2,
-                 max_frames: int = 400, no_clamp: bool = False):
+                 max_frames: int = 400, no_clamp: bool = False, allocator=None):
+        """allocator: optional (alloc(bytes) -> int device pointer or 0, release(ptr)) pair that
+        provides the handle's device memory (mh3a_create_with_allocator); it is kept alive with
+        the handle."""
         L = load()
         self.arch = arch
         self.hop = int(np.prod(arch.rates))
@@ -196,7 +211,15 @@ class Decoder:
         cfg, keep = make_config(arch, precision, max_batch, max_frames, no_clamp)
         tab, keep2 = make_table(weights)
         h = C.c_void_p()
-        _check(L.mh3a_create(C.byref(cfg), tab, len(weights), C.byref(h)), "mh3a_create")
+        self._alloc = None
+        if allocator is None:
+            _check(L.mh3a_create(C.byref(cfg), tab, len(weights), C.byref(h)), "mh3a_create")
+        else:
+            alloc_py, release_py = allocator
+            self._alloc = mh3a_allocator(ALLOC_FN(lambda n, user: alloc_py(int(n)) or None),
+                                         RELEASE_FN(lambda ptr, user: release_py(int(ptr))), None)
+            _check(L.mh3a_create_with_allocator(C.byref(cfg), tab, len(weights), C.byref(self._alloc),
+                                                C.byref(h)), "mh3a_create_with_allocator")
         self._h = h
         del keep, keep2
 

@@ -33,6 +33,8 @@
 #define MH3A_API
 #endif
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -126,6 +128,29 @@ MH3A_API void mh3a_default_config(mh3a_config* cfg);
  * architecture), MH3A_ERR_ALLOC, MH3A_ERR_CUDA.  On error *out is set to NULL. */
 MH3A_API mh3a_status mh3a_create(const mh3a_config* cfg, const mh3a_tensor* weights, int n_weights,
                         mh3a_handle** out);
+
+/* Device-memory provider for mh3a_create_with_allocator.  alloc(bytes, user) returns device
+ * memory of the current device, 256-byte aligned, or NULL on failure; release(ptr, user) gives
+ * back a pointer alloc returned.  Both are called only from mh3a_create_with_allocator (two
+ * allocations: the folded weights and the workspace) and from mh3a_destroy, on the calling host
+ * thread. */
+typedef struct {
+    void* (*alloc)(size_t bytes, void* user);
+    void (*release)(void* ptr, void* user);
+    void* user;
+} mh3a_allocator;
+
+/* mh3a_create with the handle's device memory taken from `allocator` instead of cudaMalloc
+ * (the pages have no counterpart): for hosts whose device memory is owned by another framework's
+ * allocator or pool.  allocator == NULL is mh3a_create.  A NULL alloc or release is
+ * MH3A_ERR_INVALID_ARG.  If an allocation fails (NULL, or a pointer that is not 256-byte
+ * aligned), the call returns MH3A_ERR_ALLOC, after giving back through `release` every
+ * allocation it had obtained, and sets *out to NULL; both allocations are made before any data
+ * is copied to the device.  The allocator must outlive the handle: mh3a_destroy releases
+ * through it. */
+MH3A_API mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh3a_tensor* weights,
+                                                int n_weights, const mh3a_allocator* allocator,
+                                                mh3a_handle** out);
 
 /* Decode latents (device, [B, latent_channels, N]) into a waveform (device, [B, 1, hop*N]),
  * clamped to [-1, 1] unless MH3A_FLAG_NO_CLAMP was configured.  `out` must not overlap
