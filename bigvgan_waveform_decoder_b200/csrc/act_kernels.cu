@@ -59,11 +59,13 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
     // all of the window's loads in flight at once (asynchronous copies straight to shared)
     if (!EDGE && (reinterpret_cast<uintptr_t>(xrow + t0 - 8) & 15) == 0) {
         // 16-byte copies (the window starts on a 16-byte boundary; a skewed group of 4 floats
-        // stays contiguous and 16-byte aligned in shared memory)
+        // stays contiguous and 16-byte aligned in shared memory).  Piece k of a lane is float
+        // 4 lane + 128 k of the window, at skew(4 lane) + 160 k in shared memory.
+        float* dst = xs + skew(4 * lane);
+        const float* src = xrow + t0 - 8 + 4 * lane;
 #pragma unroll
         for (int k = 0; k < (XF / 4 + 31) / 32; ++k) {
-            const int i = 4 * (lane + 32 * k);
-            if (i < XF) ptx::cp_async16(xs + skew(i), xrow + t0 - 8 + i);
+            if (4 * lane + 128 * k < XF) ptx::cp_async16(dst + 160 * k, src + 128 * k);
         }
     } else {
         // skew(lane + 32 k) = skew(lane) + 40 k
@@ -91,11 +93,14 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
         *reinterpret_cast<float4*>(trow + skew(q0 + 4 * k)) = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
     __syncthreads();
     // rows of 8 channels: skew(q + 256) = skew(q) + 320
+    ohi += t0 + tid;
+    olo += t0 + tid;
+    const int qs0 = skew(tid);
 #pragma unroll
     for (int r = 0; r < TT / NT_ACT; ++r) {
         const int q = tid + r * NT_ACT;
         if (EDGE && q >= rows) break;
-        const int qs = skew(tid) + r * (NT_ACT + NT_ACT / 4);
+        const int qs = qs0 + r * (NT_ACT + NT_ACT / 4);
         const int t = t0 + q;
         float v[8];
 #pragma unroll
@@ -109,8 +114,8 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
         split2(v[2], v[3], &hv4.y, &lv4.y);
         split2(v[4], v[5], &hv4.z, &lv4.z);
         split2(v[6], v[7], &hv4.w, &lv4.w);
-        ohi[t] = hv4;
-        olo[t] = lv4;
+        ohi[r * NT_ACT] = hv4;
+        olo[r * NT_ACT] = lv4;
     }
 }
 
@@ -123,7 +128,9 @@ __global__ void __launch_bounds__(NT_ACT, 5) k_act_split(const ActParams p) {
     const ActJob& J = p.job[blockIdx.z];
     const int L = p.L;
     const int ngroups = p.C / 8;
-    const int b = blockIdx.y / ngroups, g = blockIdx.y % ngroups;
+    // channel groups per item are a power of two at every stage width: shift and mask
+    const int b = p.g_log2 >= 0 ? (int)(blockIdx.y >> p.g_log2) : (int)blockIdx.y / ngroups;
+    const int g = (int)blockIdx.y - b * ngroups;
     const int t0 = -p.pad_l + blockIdx.x * TT;           // first output row of the tile
     const int rows = min(TT, L + p.pad_r - t0);
     const long long Lpad = (long long)L + p.pad_l + p.pad_r;
@@ -366,8 +373,11 @@ int launch_split_rows(const SplitParams& p, cudaStream_t s) {
 int launch_act_split(const ActParams& p, int njobs, cudaStream_t s) {
     if (p.C % 8 != 0 || p.L < 1 || p.pad_l < 0 || p.pad_r < 0) return -1;
     const int total = p.L + p.pad_l + p.pad_r;
-    dim3 grid((total + TT - 1) / TT, p.B * (p.C / 8), njobs);
-    return launch_dependent(k_act_split, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
+    ActParams q = p;
+    const int ng = p.C / 8;
+    q.g_log2 = (ng & (ng - 1)) == 0 ? __builtin_ctz((unsigned)ng) : -1;
+    dim3 grid((total + TT - 1) / TT, p.B * ng, njobs);
+    return launch_dependent(k_act_split, grid, dim3(NT_ACT), 0, s, q) == cudaSuccess ? 1 : -1;
 }
 
 }  // namespace mh3a

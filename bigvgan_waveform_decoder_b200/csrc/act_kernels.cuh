@@ -17,6 +17,7 @@ struct ActParams {
     ActJob job[MH3A_MAX_RESBLOCKS];
     int C, L, B;
     int pad_l, pad_r;       // zero rows before / after the sequence in the output
+    int g_log2;             // log2(C / 8) when C / 8 is a power of two, else -1 (set by the launcher)
     ActFilter filt;
 };
 

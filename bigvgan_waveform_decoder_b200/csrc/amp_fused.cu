@@ -52,6 +52,17 @@ constexpr int FW_PADO = 32;                   // margin rows of A on each side
 constexpr int FW_WO = FW_WR + 2 * FW_PADO;    // rows per channel group of A
 constexpr int FW_LAYERS = 2 * MH3A_MAX_DILATIONS;
 static_assert(FW_WR % FW_WRUN == 0, "whole warp runs per window");
+constexpr int FW_RUNS = FW_WR / FW_WRUN;      // activation runs per layer
+// The layer pipeline (see the kernel): after the activation of run k (window rows
+// [384 k, 384 k + 384)) the MMAs of tiles [fw_m_lo(k), fw_m_hi(k)) may start -- every row they
+// read, up to 157 rows past the tile's start, is written; before it, the previous layer's
+// tiles [fw_t_lo(k), fw_t_hi(k)) must be drained -- the rows this run reads (8 past its end)
+// come from them, and their MMAs are the last readers of the operand rows run k rewrites.
+static_assert(FW_RUNS == 3 && FW_MT == 9 && FW_WRUN == 384, "tile groups below are for 3 runs of 3 tiles");
+__host__ __device__ constexpr int fw_m_lo(int k) { return k == 0 ? 0 : (k == 1 ? 2 : 5); }
+__host__ __device__ constexpr int fw_m_hi(int k) { return k == 0 ? 2 : (k == 1 ? 5 : 9); }
+__host__ __device__ constexpr int fw_t_lo(int k) { return k == 0 ? 0 : (k == 1 ? 4 : 7); }
+__host__ __device__ constexpr int fw_t_hi(int k) { return k == 0 ? 4 : (k == 1 ? 7 : 9); }
 static_assert((FW_RUN * 4) % 16 == 0 && (FW_VS % 4) == 0, "16-byte aligned lane runs");
 
 // Per channel width: K-step layout of the weights and the tensor-memory columns.
@@ -80,7 +91,8 @@ struct Fw {
     static constexpr int OFF_W = OFF_AL + G * FW_WO * 16;
     static constexpr int OFF_BAR = OFF_W + 2 * WBUF;
     static constexpr int OFF_SEAM = OFF_BAR + 256;                // [NCW][8] floats
-    static constexpr int SMEM = OFF_SEAM + NCW * 8 * 4;
+    static constexpr int OFF_PAR = OFF_SEAM + NCW * 8 * 4;        // [layer][3][C] floats
+    static constexpr int SMEM = OFF_PAR + FW_LAYERS * 3 * C * 4;
     static_assert(USED <= 512, "tensor memory");
     static_assert((OFF_A % 16) == 0 && (OFF_W % 128) == 0 && (OFF_BAR % 16) == 0, "alignment");
 };
@@ -262,9 +274,30 @@ __device__ __forceinline__ void act_compute(const ActFilter& f, const ActIn& in,
     }
 }
 
+// Hand-offs between the roles are mbarriers, and every wait on them is bounded (1 s), so that a
+// defect ends the kernel with the error flag set instead of hanging it:
+//   op_full   (count: the compute warps) run k of layer l has its A operand rows written; its
+//             phase number is 3 l + k;
+//   op_taken  (count 1) the MMA warp has seen that phase: the compute warps wait for it before
+//             they complete the next one, so they never run two phases ahead;
+//   acc_full[i]  tcgen05.commit: tile i's MMAs of the layer have completed (one phase per layer);
+//   w_full / w_empty  the weight double buffer.
+// The compute warps sleep between polls (their waits are long and frequent); the only named
+// barrier is the compute warps' own (cw_sync), which they all reach in the same order.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
 template <int C>
 __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(const FwParams p) {
     using F = Fw<C>;
+    constexpr int NCW = F::NCW;
     extern __shared__ __align__(1024) uint8_t smem[];
     ptx::grid_dep_wait();   // launched as a programmatic dependent (see launch_dependent)
     float* vbuf = reinterpret_cast<float*>(smem);                      // [C][FW_VS]
@@ -274,11 +307,13 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
     uint64_t* w_full = bars;          // [2]
     uint64_t* w_empty = bars + 2;     // [2]
-    uint64_t* op_full = bars + 4;     // A operand of the current layer written
+    uint64_t* op_full = bars + 4;     // a run's A operand rows are written (phase 3 l + k)
     uint64_t* done_bar = bars + 5;    // every MMA issued has completed
     uint64_t* acc_full = bars + 6;    // [FW_MT] per tile: the layer's MMAs of the tile completed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + FW_MT);
+    uint64_t* op_taken = bars + 6 + FW_MT;   // the MMA warp has seen a phase of op_full
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + FW_MT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* par = reinterpret_cast<float*>(smem + F::OFF_PAR);         // [layer][alpha, inv_beta, bias][C]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the unit of this CTA: job (heaviest first), batch item, window
@@ -298,8 +333,9 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
             ptx::mbar_init(&w_full[i], 1);
             ptx::mbar_init(&w_empty[i], 1);
         }
-        ptx::mbar_init(op_full, 1);
         ptx::mbar_init(done_bar, 1);
+        ptx::mbar_init(op_full, NCW);
+        ptx::mbar_init(op_taken, 1);
         for (int i = 0; i < FW_MT; ++i) ptx::mbar_init(&acc_full[i], 1);
         *abort_flag = (*reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
         ptx::fence_mbar_init();
@@ -315,44 +351,50 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
 
     if (warp == 0) {
         // ------------------------------------------------------------------ MMA issuer
+        // Per layer and run k: wait for run k's operand rows, then issue the MMAs of the tiles
+        // they complete (group M_k) and commit each tile.
         constexpr uint32_t idesc1 = ptx::idesc_bf16(128, C == 8 ? 16 : 32);
         constexpr uint32_t idesc2 = ptx::idesc_bf16(128, 16);
         constexpr uint32_t b_lbo = F::BROWS * 16;
         const uint32_t ahs = ptx::smem_u32(a_hi), als = ptx::smem_u32(a_lo), ws = ptx::smem_u32(wbuf);
         bool ok = *abort_flag == 0;
-        for (int l = 0; l < nl && ok; ++l) {
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(op_full, l & 1, kFwWait));
-            if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&w_full[l & 1], (l >> 1) & 1, kFwWait));
-            if (!ok) break;
-            ptx::tc_fence_after();
-            const int d = J.dil[l];
-            const int pad = d * (J.K - 1) / 2;
-            const int KS = (C == 8) ? (J.K + 1) / 2 : J.K;
-            const uint32_t a_lbo = (C == 8) ? (uint32_t)d * 16u : (uint32_t)FW_WO * 16u;
-            const uint32_t wb = ws + (uint32_t)((l & 1) * F::WBUF);
-            for (int i = 0; i < FW_MT; ++i) {
-                const uint32_t dcol = tmem + (uint32_t)(i * F::ACC);
+        for (int l = 0; l < nl; ++l) {
+            for (int k = 0; k < FW_RUNS; ++k) {
+                const uint32_t ph = (uint32_t)(3 * l + k) & 1u;
+                if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(op_full, ph, kFwWait));
+                if (ok && k == 0) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&w_full[l & 1], (l >> 1) & 1, kFwWait));
+                if (ok && *abort_flag) ok = false;
+                if (!ok) break;
+                if (lane == 0) ptx::mbar_arrive(op_taken);
+                ptx::tc_fence_after();
+                const int d = J.dil[l];
+                const int pad = d * (J.K - 1) / 2;
+                const int KS = (C == 8) ? (J.K + 1) / 2 : J.K;
+                const uint32_t a_lbo = (C == 8) ? (uint32_t)d * 16u : (uint32_t)FW_WO * 16u;
+                const uint32_t wb = ws + (uint32_t)((l & 1) * F::WBUF);
                 for (int ks = 0; ks < KS; ++ks) {
-                    const int row = 128 * i + ((C == 8) ? 2 * ks : ks) * d - pad + FW_PADO;
-                    const uint64_t ah = ptx::desc64(ptx::desc_lo(ahs + (uint32_t)row * 16u, a_lbo));
-                    const uint64_t al = ptx::desc64(ptx::desc_lo(als + (uint32_t)row * 16u, a_lbo));
                     const uint32_t bb = wb + (uint32_t)(ks * F::KSB);
-                    if constexpr (C == 8) {
-                        const uint64_t b1 = ptx::desc64(ptx::desc_lo(bb + 128u, b_lbo));   // [B_h | B_l]
-                        const uint64_t b2 = ptx::desc64(ptx::desc_lo(bb, b_lbo));          // [0 | B_h]
-                        mma_pair_elect(dcol, ah, b1, idesc1, dcol, al, b2, idesc2, ks > 0 ? 1u : 0u);
-                    } else {
-                        const uint64_t b1 = ptx::desc64(ptx::desc_lo(bb, b_lbo));
-                        mma_pair_elect(dcol, ah, b1, idesc1, dcol + 16u, al, b1, idesc2, ks > 0 ? 1u : 0u);
+                    const uint64_t b1 = ptx::desc64(ptx::desc_lo(C == 8 ? bb + 128u : bb, b_lbo));
+                    const uint64_t b2 = ptx::desc64(ptx::desc_lo(bb, b_lbo));
+                    for (int i = fw_m_lo(k); i < fw_m_hi(k); ++i) {
+                        const uint32_t dcol = tmem + (uint32_t)(i * F::ACC);
+                        const int row = 128 * i + ((C == 8) ? 2 * ks : ks) * d - pad + FW_PADO;
+                        const uint64_t ah = ptx::desc64(ptx::desc_lo(ahs + (uint32_t)row * 16u, a_lbo));
+                        const uint64_t al = ptx::desc64(ptx::desc_lo(als + (uint32_t)row * 16u, a_lbo));
+                        if constexpr (C == 8) {
+                            // [B_h | B_l] (rows 8..23), then [0 | B_h] (rows 0..15)
+                            mma_pair_elect(dcol, ah, b1, idesc1, dcol, al, b2, idesc2, ks > 0 ? 1u : 0u);
+                        } else {
+                            mma_pair_elect(dcol, ah, b1, idesc1, dcol + 16u, al, b2, idesc2, ks > 0 ? 1u : 0u);
+                        }
                     }
                 }
-                ptx::mma_commit_elect(&acc_full[i]);
+                for (int i = fw_m_lo(k); i < fw_m_hi(k); ++i) ptx::mma_commit_elect(&acc_full[i]);
+                if (k == FW_RUNS - 1) ptx::mma_commit_elect(&w_empty[l & 1]);
             }
-            ptx::mma_commit_elect(&w_empty[l & 1]);
-            if (*abort_flag) ok = false;
-            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
         }
-        if (!ok && lane == 0) {
+        if (!ok && lane == 0 && *abort_flag == 0) {
             *abort_flag = 1;
             atomicExch(p.err, 11);
         }
@@ -368,7 +410,7 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
             for (int l = 0; l < nl && ok; ++l) {
                 const int KS = (C == 8) ? (J.K + 1) / 2 : J.K;
                 const uint32_t bytes = (uint32_t)(KS * F::KSB);
-                if (!ptx::mbar_wait(&w_empty[l & 1], ((l >> 1) & 1) ^ 1, kFwWait) || *abort_flag) {
+                if (!mbar_wait_sleepy(&w_empty[l & 1], ((l >> 1) & 1) ^ 1, kFwWait) || *abort_flag) {
                     ok = false;
                     break;
                 }
@@ -376,36 +418,51 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
                 ptx::bulk_g2s(wbuf + (l & 1) * F::WBUF, J.w[l], bytes, &w_full[l & 1]);
                 issued = l + 1;
             }
-            if (!ok) {
+            if (!ok && *abort_flag == 0) {
                 *abort_flag = 1;
                 atomicExch(p.err, 12);
             }
             // the copies in flight land before the CTA may exit
             for (int l = (issued > 2 ? issued - 2 : 0); l < issued; ++l)
-                ptx::mbar_wait(&w_full[l & 1], (l >> 1) & 1, kFwWait);
+                mbar_wait_sleepy(&w_full[l & 1], (l >> 1) & 1, kFwWait);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ compute warps
-        constexpr int NCW = F::NCW;
         const int cw = warp - 2;
         const int ct = threadIdx.x - 64;
         const int q4 = warp & 3;                   // tensor-memory lane quarter of this warp
         const int sub = cw >> 2, nsub = NCW / 4;   // this warp's share of the tiles
-        bool ok = *abort_flag == 0;
+        const bool edge = r_lo > 0 || r_hi < FW_WR;
         // zero the operand margins once (read only by rows that are never written out)
         for (int i = ct; i < 2 * F::G * FW_WO; i += NCW * 32) {
             uint8_t* base = (i < F::G * FW_WO) ? a_hi : a_lo;
             const int k = i % (F::G * FW_WO);
             *reinterpret_cast<uint4*>(base + (size_t)k * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
+        // per-layer activation and bias parameters
+        for (int i = ct; i < nl * 3 * C; i += NCW * 32) {
+            const int l = i / (3 * C), k = (i / C) % 3, c = i % C;
+            const float* src = k == 0 ? J.alpha[l] : (k == 1 ? J.inv_beta[l] : J.bias[l]);
+            par[i] = __ldg(src + c);
+        }
         // the input window (replicate padding: the time index is clamped into the sequence)
         {
             const float* xb = p.x + (long long)b * C * L;
-            for (int i = ct; i < C * FW_VS; i += NCW * 32) {
-                const int c = i / FW_VS, r = i - c * FW_VS - FW_VM;
-                const int t = min(max(tw + r, 0), L - 1);
-                ptx::cp_async4(vbuf + i, xb + (long long)c * L + t);
+            const bool vec = !edge && tw >= FW_VM && tw + FW_WR + FW_VM <= L && (L & 3) == 0 && (tw & 3) == 0 &&
+                             (reinterpret_cast<uintptr_t>(p.x) & 15) == 0;
+            if (vec) {
+                constexpr int Q = FW_VS / 4;   // 16-byte pieces per channel row
+                for (int i = ct; i < C * Q; i += NCW * 32) {
+                    const int c = i / Q, q = i - c * Q;
+                    ptx::cp_async16(vbuf + c * FW_VS + 4 * q, xb + (long long)c * L + tw - FW_VM + 4 * q);
+                }
+            } else {
+                for (int i = ct; i < C * FW_VS; i += NCW * 32) {
+                    const int c = i / FW_VS, r = i - c * FW_VS - FW_VM;
+                    const int t = min(max(tw + r, 0), L - 1);
+                    ptx::cp_async4(vbuf + i, xb + (long long)c * L + t);
+                }
             }
             ptx::cp_async_commit();
             ptx::cp_async_wait_all();
@@ -420,34 +477,83 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
             x_st<C>(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(F::XCOL0 + i * C), xv);
         }
         tmem_wait_st();
-        const bool edge = r_lo > 0 || r_hi < FW_WR;
-        for (int l = 0; l < nl; ++l) {
-            // ---- activation of v into the A operand
-            if (edge) {
-                // replicate padding of the activation's input: rows outside the sequence take
-                // the end samples (their current contents are not the signal there)
-                for (int i = ct; i < C * FW_VS; i += NCW * 32) {
-                    const int c = i / FW_VS, r = i - c * FW_VS - FW_VM;
-                    if (r < r_lo) vbuf[i] = vbuf[c * FW_VS + FW_VM + r_lo];
-                    else if (r >= r_hi) vbuf[i] = vbuf[c * FW_VS + FW_VM + r_hi - 1];
+        for (int l = 0; l <= nl; ++l) {
+            const float* pl = par + l * 3 * C;                      // this layer's activation
+            const float* pp = par + (l > 0 ? l - 1 : 0) * 3 * C;    // the previous layer's bias
+            for (int k = 0; k < FW_RUNS; ++k) {
+                // ---- epilogue of the previous layer's tiles in group T_k
+                if (l > 0) {
+                    const bool second = ((l - 1) & 1) != 0;
+                    for (int i = fw_t_lo(k); i < fw_t_hi(k); ++i) {
+                        if (i % nsub != sub) continue;
+                        bool got = *abort_flag == 0 && mbar_wait_sleepy(&acc_full[i], (uint32_t)(l - 1) & 1u, kFwWait);
+                        got = __all_sync(0xffffffffu, got);
+                        if (!got) {
+                            if (lane == 0 && *abort_flag == 0) {
+                                *abort_flag = 1;
+                                atomicExch(p.err, 13);
+                            }
+                            continue;
+                        }
+                        ptx::tc_fence_after();
+                        const int r = 128 * i + 32 * q4 + lane;
+                        const uint32_t lq = (uint32_t)(32 * q4) << 16;
+                        float y[C];
+                        if constexpr (C == 8) {
+                            float v[16];
+                            ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) y[c] = (v[c] + v[8 + c]) + pp[2 * C + c];
+                        } else {
+                            float v0[16], v1[16];
+                            ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v0);
+                            ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC + 16), v1);
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) y[c] = (v0[c] + v1[c]) + pp[2 * C + c];
+                        }
+                        if (second) {
+                            float xo[C];
+                            const uint32_t xa = tmem + lq + (uint32_t)(F::XCOL0 + i * C);
+                            x_ld<C>(xa, xo);
+#pragma unroll
+                            for (int c = 0; c < C; ++c) y[c] = xo[c] + y[c];
+                            if (l < nl) x_st<C>(xa, y);
+                        }
+#pragma unroll
+                        for (int c = 0; c < C; ++c) vbuf[c * FW_VS + FW_VM + r] = y[c];
+                    }
+                    tmem_wait_st();
                 }
-                cw_sync(NCW);
-            }
-            // one channel per warp, its runs in order (see act_load)
-            static_assert(F::NCW == C, "one compute warp per channel");
-            {
-                const int c = cw;
-                float* vr = vbuf + c * FW_VS + FW_VM;
-                float* seam = reinterpret_cast<float*>(smem + F::OFF_SEAM) + cw * 8;
-                const float al = __ldg(J.alpha[l] + c), ib = __ldg(J.inv_beta[l] + c);
-#pragma unroll 1
-                for (int k = 0; k < FW_WR / FW_WRUN; ++k) {
-                    const int rw = k * FW_WRUN;
+                if (l == nl) continue;
+                const bool ok = *abort_flag == 0;
+                const int rw = k * FW_WRUN;
+                cw_sync(NCW);   // the epilogue rows this run reads are written
+                if (edge) {
+                    // replicate padding of the activation's input over this run's input rows:
+                    // rows outside the sequence take the end samples (only sources this run's
+                    // epilogue groups have written are used; rows whose source lies later are
+                    // outside the sequence on every row this run outputs)
+                    const int lo = (k == 0) ? rw - FW_VM : rw, hi = rw + FW_WRUN + FW_VM;
+                    for (int i = ct; i < C * (hi - lo); i += NCW * 32) {
+                        const int c = i / (hi - lo), r = lo + i - c * (hi - lo);
+                        float* vr = vbuf + c * FW_VS + FW_VM;
+                        if (r < r_lo && r_lo < hi) vr[r] = vr[r_lo];
+                        else if (r >= r_hi && r_hi - 1 >= lo) vr[r] = vr[r_hi - 1];
+                    }
+                    cw_sync(NCW);
+                }
+                // ---- activation of run k, one channel per warp (see act_load)
+                static_assert(F::NCW == C, "one compute warp per channel");
+                {
+                    const int c = cw;
+                    float* vr = vbuf + c * FW_VS + FW_VM;
+                    float* seam = reinterpret_cast<float*>(smem + F::OFF_SEAM) + cw * 8;
+                    const float al = pl[c], ib = pl[C + c];
                     ActIn in;
                     act_load(vr, k > 0 ? seam : nullptr, rw, in);
                     __syncwarp();
                     // the next run's left input rows, before this run overwrites them
-                    if (k + 1 < FW_WR / FW_WRUN && lane < 8) seam[lane] = vr[rw + FW_WRUN - 8 + lane];
+                    if (k + 1 < FW_RUNS && lane < 8) seam[lane] = vr[rw + FW_WRUN - 8 + lane];
                     __syncwarp();
                     if (ok) {
                         float a[FW_RUN];
@@ -461,92 +567,54 @@ __global__ void __launch_bounds__(Fw<C>::NTHR, (C == 8) ? 2 : 1) k_amp_fused(con
                             *reinterpret_cast<float4*>(dst + 4 * q) =
                                 make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
                     }
-                    __syncwarp();
                 }
-            }
-            cw_sync(NCW);
-            // transposing split: rows of 8 channels, heads and tails; zeros outside the sequence
-            if (ok) {
-                for (int i = ct; i < F::G * FW_WR; i += NCW * 32) {
-                    const int g = i / FW_WR, r = i - g * FW_WR;
-                    float v[8];
+                cw_sync(NCW);
+                // transposing split of run k's rows: rows of 8 channels, heads and tails; zeros
+                // outside the sequence
+                if (ok) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) v[c] = vbuf[(8 * g + c) * FW_VS + FW_VM + r];
-                    uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;
-                    if (r >= r_lo && r < r_hi) {
-                        actm::split2(v[0], v[1], &hv.x, &lv.x);
-                        actm::split2(v[2], v[3], &hv.y, &lv.y);
-                        actm::split2(v[4], v[5], &hv.z, &lv.z);
-                        actm::split2(v[6], v[7], &hv.w, &lv.w);
+                    for (int g = 0; g < F::G; ++g) {
+                        const float* vg = vbuf + (8 * g) * FW_VS + FW_VM;
+                        uint8_t* hg = a_hi + ((size_t)g * FW_WO + FW_PADO) * 16;
+                        uint8_t* lg = a_lo + ((size_t)g * FW_WO + FW_PADO) * 16;
+                        for (int r = rw + ct; r < rw + FW_WRUN; r += NCW * 32) {
+                            float v[8];
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) v[c] = vg[c * FW_VS + r];
+                            uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = hv;
+                            if (r >= r_lo && r < r_hi) {
+                                actm::split2(v[0], v[1], &hv.x, &lv.x);
+                                actm::split2(v[2], v[3], &hv.y, &lv.y);
+                                actm::split2(v[4], v[5], &hv.z, &lv.z);
+                                actm::split2(v[6], v[7], &hv.w, &lv.w);
+                            }
+                            *reinterpret_cast<uint4*>(hg + r * 16) = hv;
+                            *reinterpret_cast<uint4*>(lg + r * 16) = lv;
+                        }
                     }
-                    const size_t off = ((size_t)g * FW_WO + FW_PADO + r) * 16;
-                    *reinterpret_cast<uint4*>(a_hi + off) = hv;
-                    *reinterpret_cast<uint4*>(a_lo + off) = lv;
                 }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            cw_sync(NCW);
-            if (ct == 0) ptx::mbar_arrive(op_full);
-            // ---- epilogue of the layer's conv, tile by tile as the MMAs complete
-            const bool second = (l & 1) != 0;
-            float bias[C];
-#pragma unroll
-            for (int c = 0; c < C; ++c) bias[c] = __ldg(J.bias[l] + c);
-            for (int i = sub; i < FW_MT; i += nsub) {
-                if (ok && *abort_flag) ok = false;
-                if (ok && !ptx::mbar_wait(&acc_full[i], l & 1, kFwWait)) {
-                    ok = false;
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                // complete phase 3 l + k of op_full, once the MMA warp has seen the previous one
+                const int ph = 3 * l + k;
+                bool seen = ph == 0 || *abort_flag != 0 ||
+                            mbar_wait_sleepy(op_taken, (uint32_t)(ph - 1) & 1u, kFwWait);
+                seen = __all_sync(0xffffffffu, seen);
+                if (!seen && lane == 0 && *abort_flag == 0) {
                     *abort_flag = 1;
-                    atomicExch(p.err, 13);
+                    atomicExch(p.err, 15);
                 }
-                if (!__all_sync(0xffffffffu, ok)) {
-                    ok = false;
-                    continue;
-                }
-                ptx::tc_fence_after();
-                const int r = 128 * i + 32 * q4 + lane;
-                const uint32_t lq = (uint32_t)(32 * q4) << 16;
-                float y[C];
-                if constexpr (C == 8) {
-                    float v[16];
-                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) y[c] = (v[c] + v[8 + c]) + bias[c];
-                } else {
-                    float v0[16], v1[16];
-                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC), v0);
-                    ptx::tmem_ld16(tmem + lq + (uint32_t)(i * F::ACC + 16), v1);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) y[c] = (v0[c] + v1[c]) + bias[c];
-                }
-                if (second) {
-                    float xo[C];
-                    const uint32_t xa = tmem + lq + (uint32_t)(F::XCOL0 + i * C);
-                    x_ld<C>(xa, xo);
-#pragma unroll
-                    for (int c = 0; c < C; ++c) y[c] = xo[c] + y[c];
-                    if (l + 1 < nl) x_st<C>(xa, y);
-                }
-#pragma unroll
-                for (int c = 0; c < C; ++c) vbuf[c * FW_VS + FW_VM + r] = y[c];
+                if (lane == 0) ptx::mbar_arrive(op_full);
             }
-            tmem_wait_st();
-            ptx::tc_fence_before();
-            cw_sync(NCW);
         }
+        cw_sync(NCW);
         // ---- the window's output rows
-        if (ok) {
+        if (*abort_flag == 0) {
             const int n_out = min(J.T, L - t0);
             float* ob = J.out + (long long)b * C * L + t0;
-            for (int i = ct; i < C * n_out; i += NCW * 32) {
-                const int c = i / n_out, k = i - c * n_out;
-                ob[(long long)c * L + k] = vbuf[c * FW_VS + FW_VM + J.H + k];
-            }
-        }
-        if (!ok) {
-            *abort_flag = 1;
-            atomicExch(p.err, 14);
+#pragma unroll
+            for (int c = 0; c < C; ++c)
+                for (int k = ct; k < n_out; k += NCW * 32) ob[(long long)c * L + k] = vbuf[c * FW_VS + FW_VM + J.H + k];
         }
     }
     ptx::grid_dep_launch();
@@ -580,10 +648,12 @@ float bf16_bits_value(uint16_t h) {
 
 }  // namespace
 
+// Rows of receptive field per side of one residual block, rounded up to a multiple of 4 so that
+// windows start on 16-byte boundaries of a sequence whose length is a multiple of 4.
 int fused_halo(int K, const int* dil, int nd) {
     int H = 0;
     for (int m = 0; m < nd; ++m) H += 5 + dil[m] * (K - 1) / 2 + 5 + (K - 1) / 2;
-    return H;
+    return (H + 3) / 4 * 4;
 }
 
 bool fused_stage_supported(int C, const mh3a_config& c) {
