@@ -628,6 +628,7 @@ mh3a_status amp_stage_into(mh3a_handle* h, const float* x, int B, int L, int sta
     const mh3a_config& c = h->cfg;
     const int C = stage_channels(c, stage);
     const int nrb = c.n_resblocks;
+    ConvParams layers[2 * MH3A_MAX_DILATIONS];
     for (int m = 0; m < c.n_dilations; ++m) {
         for (int half = 0; half < 2; ++half) {
             ConvParams p{};
@@ -654,14 +655,24 @@ mh3a_status amp_stage_into(mh3a_handle* h, const float* x, int B, int L, int sta
                 J.dil = d;
                 J.pad = d * (k - 1) / 2;
             }
-            // the fused tensor-core kernel (activation computed in its own producer warps) needs
-            // no operand buffers beyond X and T; it serves widths of 32 channels and more
+            if (h->stage_fused[stage]) {
+                layers[2 * m + half] = p;   // the fused stage kernel, launched below
+                continue;
+            }
+            // the fused tensor-core layer kernel (activation computed in its own producer warps)
+            // needs no operand buffers beyond X and T; it serves widths of 32 channels and more
             const int n = (h->stage_tc[stage] && C >= 32)
                               ? launch_conv_tc(p, nrb, h->tc[stage], m, half, s, h->dev_err)
                               : launch_conv_simt(p, nrb, /*act=*/true, /*mean3=*/false, s);
             mh3a_status st = counted(h, n);
             if (st) return st;
         }
+    }
+    if (h->stage_fused[stage]) {
+        // the kernel mh3a_amp_stage and the decode run for this stage: it needs no scratch but
+        // the block outputs X
+        mh3a_status st = counted(h, launch_amp_fused(layers, 2 * c.n_dilations, nrb, h->tc[stage], x, s, h->dev_err));
+        if (st) return st;
     }
     Mean3Params mp{X[0], X[1], X[2], out, (long long)B * C * L, 0};
     mp.vec4 = ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(X[0]) |

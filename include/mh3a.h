@@ -178,7 +178,14 @@ MH3A_API mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L
  * once at start-up (it may pass max_batch = max_frames = 1 to keep the handle's own workspace
  * small) and then runs stages through this call, which allocates nothing.
  *
- * Arguments, results and status codes are those of mh3a_amp_stage.  The six intermediate
+ * Arguments and status codes are those of mh3a_amp_stage.  The results agree with
+ * mh3a_amp_stage's within the parity tolerance of the handle's precision, and are identical to
+ * them bit for bit where this call runs the same kernel: at a stage that the decode runs as one
+ * fused kernel (8 channels in MH3A_BF16X3 mode), which needs no scratch beyond the block
+ * outputs.  At the other stages the decode's tensor-core path stages the activation through
+ * operand arrays in the workspace; this call instead runs a layer kernel that computes the
+ * activation inside the conv (32 channels and wider) or the fp32 CUDA-core kernels (narrower),
+ * so its low-order bits differ.  The six intermediate
  * [B, C, L] buffers of the stage live in one fixed array of MH3A_STATIC_SCRATCH_BYTES in the
  * library's device image: the CUDA runtime places it when it loads the library's code onto a
  * GPU, and every GPU that loads the library holds it until the process exits.  B * C * L must

@@ -4,7 +4,8 @@ framework's budget).  It keeps its intermediate buffers in a fixed array inside 
 device image instead of the handle's workspace.
 
 Checked through the C ABI against the workspace entry point mh3a_amp_stage, on two calls in a
-row with different inputs, within the parity tolerances the other GPU tests use.  The handle
+row with different inputs, within the parity tolerances the other GPU tests use, and bit for bit
+at the stage where both run the same fused kernel.  The handle
 used for the static calls is created with the smallest workspace (max_batch = max_frames = 1),
 so those calls cannot be reading the handle's workspace.  This file is collected last.
 """
@@ -24,6 +25,7 @@ pytestmark = pytest.mark.gpu
 
 TOL = {Bd.MH3A_FP32: (1e-5, None), Bd.MH3A_BF16X3: (2e-3, 1e-2)}
 LIMIT = 2796160  # MH3A_STATIC_SCRATCH_MAX_ELEMS
+FUSED_STAGES = (6,)  # stages the decode runs as one fused kernel in BF16X3 mode (8 channels)
 
 
 def _static_fn():
@@ -74,6 +76,9 @@ def test_static_scratch_stage_matches_workspace_stage(precision):
                 small.check_device_error()
                 ref_dec.check_device_error()
                 _close(out, ref, precision, f"stage {stage} call {call}")
+                if precision == Bd.MH3A_BF16X3 and stage in FUSED_STAGES:
+                    # the same fused kernel as mh3a_amp_stage: identical bits
+                    assert torch.equal(out, ref), f"stage {stage} call {call}: not bit-identical"
         # beyond the static limit: rejected on the host with a clear message, output untouched
         C0 = arch.stage_channels(0)
         L_big = LIMIT // C0 + 1
