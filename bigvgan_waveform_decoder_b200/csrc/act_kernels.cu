@@ -119,9 +119,10 @@ __device__ __forceinline__ void act_tile(const ActParams& p, const ActJob& J, fl
     }
 }
 
-// grid: x = row tiles over [-pad_l, L + pad_r), y = B * C / 8 (item, group), z = job.  Five
-// blocks per SM (48 registers, a few spilled to L1) issue better than four blocks at 64.
-__global__ void __launch_bounds__(NT_ACT, 5) k_act_split(const ActParams p) {
+// grid: x = row tiles over [-pad_l, L + pad_r), y = B * C / 8 (item, group), z = job.  With the
+// packed fp32x2 SnakeBeta and decimation, four blocks per SM at 64 registers (no spills) issue
+// slightly better than five at 48 (which spill a few registers to L1).
+__global__ void __launch_bounds__(NT_ACT, 4) k_act_split(const ActParams p) {
     ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
     ptx::grid_dep_launch();
     __shared__ __align__(16) float buf[SMEM_FLOATS];

@@ -76,6 +76,33 @@ __device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv,
     }
 }
 
+// SnakeBeta values J and J + 1 (J even) as one packed pair: the two upsampled values, then
+// alpha u, sin, its square and the final fma as fp32x2 operations where the hardware has them.
+template <int J>
+__device__ __forceinline__ void snake_pair(const ActFilter& f, const float* xv, float2 al2, float2 ib2, float* s) {
+    static_assert(J % 2 == 0, "pairs start on even indices");
+    float ua = 0.f, ub = 0.f;
+#pragma unroll
+    for (int k = 0; k < 6; ++k) {
+        ua = fmaf(f.up[2 * k], xv[8 + J / 2 - k], ua);        // J even: odd phase
+        ub = fmaf(f.up[2 * k + 1], xv[8 + J / 2 - k], ub);    // J + 1 odd: even phase
+    }
+    const float2 u2 = make_float2(ua, ub);
+    const float2 t2 = __fmul2_rn(al2, u2);
+    const float2 sn = make_float2(__sinf(t2.x), __sinf(t2.y));
+    const float2 r2 = __ffma2_rn(__fmul2_rn(sn, sn), ib2, u2);
+    s[J] = r2.x;
+    s[J + 1] = r2.y;
+}
+
+template <int J0, int J1>
+__device__ __forceinline__ void snake_pairs(const ActFilter& f, const float* xv, float2 al2, float2 ib2, float* s) {
+    if constexpr (J0 < J1) {
+        snake_pair<J0>(f, xv, al2, ib2, s);
+        snake_pairs<J0 + 2, J1>(f, xv, al2, ib2, s);
+    }
+}
+
 // Outputs a[k] = act(x)[tw + RUN lane + k] of one channel (RUN even).  xs: the skewed window,
 // logical index i <-> x[tw - 8 + i], at least 32 RUN + 16 floats, staged with the sequence's
 // replicate padding when EDGE.  EDGE also substitutes the end values for SnakeBeta positions
@@ -107,7 +134,11 @@ __device__ __forceinline__ void act_lane(const ActFilter& f, const float* xs, fl
         }
     }
     float s[NS];
-    snake_range<5, 5 + 2 * RUN>(f, xv, al, ib, s);     // the lane's own 2 RUN values
+    // the lane's own 2 RUN values, s[5 .. 2 RUN + 4]: the interior pairs (s[2m], s[2m + 1]) go
+    // through SnakeBeta as packed fp32x2 operations (the same rounding as the scalar form)
+    s[5] = snake_at<5>(f, xv, al, ib);
+    snake_pairs<6, 2 * RUN + 4>(f, xv, make_float2(al, al), make_float2(ib, ib), s);
+    s[2 * RUN + 4] = snake_at<2 * RUN + 4>(f, xv, al, ib);
     // The 5 values left of lane 0's run and right of lane 31's run: lanes 0-4 and 5-9 form one
     // each (value j of lane 0's window, resp. j = 2 RUN + 5 .. 2 RUN + 9 of lane 31's).
     float hv = 0.f;
@@ -141,12 +172,15 @@ __device__ __forceinline__ void act_lane(const ActFilter& f, const float* xs, fl
 #pragma unroll
         for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
     }
+    // decimation: even and odd taps as the two halves of packed fp32x2 FMAs on the pairs
+    // (s[2m], s[2m + 1]), then one add
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
-        float v = 0.f;
+        float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(f.down[j], s[2 * i + j], v);
-        a[i] = v;
+        for (int q = 0; q < kFilterTaps / 2; ++q)
+            v = __ffma2_rn(make_float2(f.down[2 * q], f.down[2 * q + 1]), make_float2(s[2 * i + 2 * q], s[2 * i + 2 * q + 1]), v);
+        a[i] = v.x + v.y;
     }
 }
 
