@@ -81,13 +81,14 @@ __device__ __forceinline__ void snake_range(const ActFilter& f, const float* xv,
 template <int J>
 __device__ __forceinline__ void snake_pair(const ActFilter& f, const float* xv, float2 al2, float2 ib2, float* s) {
     static_assert(J % 2 == 0, "pairs start on even indices");
-    float ua = 0.f, ub = 0.f;
+    // J even reads the odd phase taps f[2k], J + 1 the even phase taps f[2k + 1], both at the
+    // same input sample: one packed fma per tap pair
+    float2 u2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < 6; ++k) {
-        ua = fmaf(f.up[2 * k], xv[8 + J / 2 - k], ua);        // J even: odd phase
-        ub = fmaf(f.up[2 * k + 1], xv[8 + J / 2 - k], ub);    // J + 1 odd: even phase
+        const float xk = xv[8 + J / 2 - k];
+        u2 = __ffma2_rn(make_float2(f.up[2 * k], f.up[2 * k + 1]), make_float2(xk, xk), u2);
     }
-    const float2 u2 = make_float2(ua, ub);
     const float2 t2 = __fmul2_rn(al2, u2);
     const float2 sn = make_float2(__sinf(t2.x), __sinf(t2.y));
     const float2 r2 = __ffma2_rn(__fmul2_rn(sn, sn), ib2, u2);
