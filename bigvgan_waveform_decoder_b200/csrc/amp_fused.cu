@@ -228,19 +228,11 @@ __device__ __forceinline__ void act_compute(const ActFilter& f, const ActIn& in,
     const int lane = threadIdx.x & 31;
     const int rs = rw + RUN * lane;
     float s[NS];
-    // own values: s[5 + i] at local 2x index 2 rs + i
-#pragma unroll
-    for (int i = 0; i < 2 * RUN; ++i) {
-        float u = 0.f;
-        if (i % 2 == 0) {
-#pragma unroll
-            for (int q = 0; q < 6; ++q) u = fmaf(f.up[2 * q + 1], in.xv[i / 2 + 10 - q], u);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 6; ++q) u = fmaf(f.up[2 * q], in.xv[(i - 1) / 2 + 11 - q], u);
-        }
-        s[5 + i] = fmaf(actm::sin_sq_fast(al, u), ib, u);
-    }
+    // own values: s[5 + i] at local 2x index 2 rs + i (xv[k] = v[rs - 8 + k], the layout of the
+    // standalone kernel's lane routine): the two ends scalar, the interior pairs packed
+    s[5] = actm::snake_at<5>(f, in.xv, al, ib);
+    actm::snake_pairs<6, 2 * RUN + 4>(f, in.xv, make_float2(al, al), make_float2(ib, ib), s);
+    s[2 * RUN + 4] = actm::snake_at<2 * RUN + 4>(f, in.xv, al, ib);
     float hv = 0.f;
     if (lane < 10) hv = snake_from6(f, in.hq, halo_n(lane, rw), al, ib);
 #pragma unroll
@@ -265,12 +257,14 @@ __device__ __forceinline__ void act_compute(const ActFilter& f, const ActIn& in,
 #pragma unroll
         for (int j = 0; j < NS; ++j) s[j] = (j < j0) ? sf : ((j > je) ? sl : s[j]);
     }
+    // decimation: even and odd taps as the halves of packed fma chains, then one add
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
-        float v = 0.f;
+        float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < kFilterTaps; ++j) v = fmaf(f.down[j], s[2 * i + j], v);
-        a[i] = v;
+        for (int q = 0; q < kFilterTaps / 2; ++q)
+            v = __ffma2_rn(make_float2(f.down[2 * q], f.down[2 * q + 1]), make_float2(s[2 * i + 2 * q], s[2 * i + 2 * q + 1]), v);
+        a[i] = v.x + v.y;
     }
 }
 
