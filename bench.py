@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--precision", choices=["bf16x3", "fp32"], default="bf16x3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every decode directly instead of replaying its CUDA graph")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the single-stage and batched-decode figures")
     ap.add_argument("--ref-sample-frames", type=int, default=200,
@@ -248,6 +250,7 @@ def extra_batched(arch_w, Bd, flush, stream, dev, steps: int) -> dict:
     arch, w, z = arch_w
     B, _, N = z.shape
     dec = Bd.Decoder(arch, w, precision=Bd.MH3A_BF16X3, max_batch=B, max_frames=N)
+    dec.set_graph_mode(True)
     x = torch.from_numpy(z).to(dev)
     out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
     for _ in range(2):
@@ -286,7 +289,13 @@ def run_ours(args):
     x = torch.from_numpy(z).to(dev)
     out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
     flush = torch.empty(FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
-    stream = torch.cuda.current_stream()
+    # A stream of our own: the legacy default stream cannot be captured, so decodes on it never
+    # replay a graph.  torch's fills of the L2 flush buffer run on it too.
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    if not args.no_graph:
+        dec.set_graph_mode(True)   # the first warm-up decode captures, the rest replay
     audio_s = B * N / 40.0
     n_stages = len(arch.rates)
 
@@ -408,7 +417,7 @@ def run_ours(args):
         "config": {"workload": f"decode B={B} N={N} (10 s stereo, 2 x 320000 samples) per GPU",
                    "global_batch": B * world, "latent_frames": N, "replicas": world,
                    "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)",
-                   "statistic": "median step"},
+                   "statistic": "median step", "cuda_graph": not args.no_graph},
         "roofline": roofline,
         "roofline_activation": roofline_act,
         "e2e": {"value": e2e_value, "unit": UNIT,

@@ -24,7 +24,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "sh
 
 EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_create_with_allocator", "mh3a_decode",
            "mh3a_decode_host",
-           "mh3a_amp_stage", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
+           "mh3a_amp_stage", "mh3a_set_graph_mode", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
            "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error",
            "mh3a_stage_uses_tensor_cores", "mh3a_segment_uses_tensor_cores",
            "mh3a_check_device_error")
@@ -104,6 +104,8 @@ def load():
     L.mh3a_decode_host.restype = C.c_int
     L.mh3a_amp_stage.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, vp, vp]
     L.mh3a_amp_stage.restype = C.c_int
+    L.mh3a_set_graph_mode.argtypes = [vp, C.c_int]
+    L.mh3a_set_graph_mode.restype = C.c_int
     L.mh3a_set_profiling.argtypes = [vp, C.c_int]
     L.mh3a_set_profiling.restype = C.c_int
     L.mh3a_set_kernel_profiling.argtypes = [vp, C.c_int]
@@ -256,6 +258,10 @@ class Decoder:
         _check(load().mh3a_amp_stage(self._h, x.data_ptr(), B, Lx, stage, out.data_ptr(),
                                      _stream_ptr(stream)), "mh3a_amp_stage")
         return out
+
+    def set_graph_mode(self, on: bool):
+        """Replay each (B, N, input, output) decode from a CUDA graph captured on first use."""
+        _check(load().mh3a_set_graph_mode(self._h, 1 if on else 0), "mh3a_set_graph_mode")
 
     def set_profiling(self, on: bool):
         _check(load().mh3a_set_profiling(self._h, 1 if on else 0), "mh3a_set_profiling")

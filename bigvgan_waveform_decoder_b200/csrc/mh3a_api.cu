@@ -147,6 +147,19 @@ struct mh3a_handle {
     int kev_rec = -1;                       // the stage the last decode recorded
     bool kev_fused = false;                 // it was a fused stage: one launch, kev[0][0..1]
     long long launches = 0;
+    // graph replay (mh3a_set_graph_mode): one captured decode per (B, N, input, output)
+    struct GraphEntry {
+        int B = 0, N = 0;
+        const float* in = nullptr;
+        float* out = nullptr;
+        cudaGraphExec_t exec = nullptr;
+        long long launches = 0;          // kernels one replay launches
+        unsigned long long used = 0;     // last use, for replacement
+    };
+    static constexpr int kGraphSlots = 4;
+    bool graph_mode = false;
+    GraphEntry graphs[kGraphSlots];
+    unsigned long long graph_tick = 0;
 };
 
 namespace {
@@ -735,6 +748,8 @@ void mh3a_destroy(mh3a_handle* h) {
     cudaGetDevice(&prev);
     cudaSetDevice(h->device);
     cudaDeviceSynchronize();
+    for (auto& g : h->graphs)
+        if (g.exec) cudaGraphExecDestroy(g.exec);
     for (auto& e : h->ev)
         if (e) cudaEventDestroy(e);
     for (auto& li : h->kev)
@@ -936,10 +951,83 @@ mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh3a_tensor
     return MH3A_OK;
 }
 
+namespace {
+
+// A decode through the graph cache: the first call for a (B, N, input, output) captures the
+// decode's launches on `s` and instantiates them; every call launches the instantiated graph.
+// Streams that cannot be captured (the legacy default stream) and streams the caller is already
+// capturing run the launches directly.
+mh3a_status decode_dispatch(mh3a_handle* h, const float* in, int B, int N, float* out, cudaStream_t s) {
+    const bool special = s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread;
+    if (!h->graph_mode || h->profiling || h->kprof_stage >= 0 || special) return run_decode(h, in, B, N, out, s);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    CK_CUDA(cudaStreamIsCapturing(s, &cs), "cudaStreamIsCapturing");
+    if (cs != cudaStreamCaptureStatusNone) return run_decode(h, in, B, N, out, s);
+    mh3a_handle::GraphEntry* e = nullptr;
+    for (auto& g : h->graphs)
+        if (g.exec && g.B == B && g.N == N && g.in == in && g.out == out) e = &g;
+    if (!e) {
+        // a free slot, else the least recently used one
+        e = &h->graphs[0];
+        for (auto& g : h->graphs) {
+            if (!g.exec) { e = &g; break; }
+            if (g.used < e->used) e = &g;
+        }
+        if (e->exec) {
+            // its last replay may still be running on some stream
+            CK_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+            CK_CUDA(cudaGraphExecDestroy(e->exec), "cudaGraphExecDestroy");
+            *e = mh3a_handle::GraphEntry{};
+        }
+        CK_CUDA(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "cudaStreamBeginCapture");
+        const long long l0 = h->launches;
+        const mh3a_status st = run_decode(h, in, B, N, out, s);
+        cudaGraph_t graph = nullptr;
+        const cudaError_t ce = cudaStreamEndCapture(s, &graph);
+        const long long nl = h->launches - l0;
+        h->launches = l0;   // the capture itself launched nothing
+        if (st != MH3A_OK || ce != cudaSuccess) {
+            if (graph) cudaGraphDestroy(graph);
+            return st != MH3A_OK ? st : cuda_fail(ce, "cudaStreamEndCapture");
+        }
+        cudaGraphExec_t exec = nullptr;
+        const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (ie != cudaSuccess) return cuda_fail(ie, "cudaGraphInstantiate");
+        e->B = B;
+        e->N = N;
+        e->in = in;
+        e->out = out;
+        e->exec = exec;
+        e->launches = nl;
+    }
+    e->used = ++h->graph_tick;
+    CK_CUDA(cudaGraphLaunch(e->exec, s), "cudaGraphLaunch");
+    h->launches += e->launches;
+    return MH3A_OK;
+}
+
+}  // namespace
+
+mh3a_status mh3a_set_graph_mode(mh3a_handle* h, int enable) {
+    if (!h) return MH3A_ERR_INVALID_ARG;
+    if (!enable) {
+        CK_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");   // no replay still running
+        for (auto& g : h->graphs) {
+            if (g.exec) {
+                CK_CUDA(cudaGraphExecDestroy(g.exec), "cudaGraphExecDestroy");
+            }
+            g = mh3a_handle::GraphEntry{};
+        }
+    }
+    h->graph_mode = enable != 0;
+    return MH3A_OK;
+}
+
 mh3a_status mh3a_decode(mh3a_handle* h, const float* latents, int B, int N, float* out, void* stream) {
     if (!h || !latents || !out) return MH3A_ERR_INVALID_ARG;
     if (B < 1 || N < 1 || B > h->cfg.max_batch || N > h->cfg.max_frames) return MH3A_ERR_SHAPE;
-    return run_decode(h, latents, B, N, out, (cudaStream_t)stream);
+    return decode_dispatch(h, latents, B, N, out, (cudaStream_t)stream);
 }
 
 mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, int N, float* out_host,
@@ -950,7 +1038,7 @@ mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, i
     const size_t in_bytes = (size_t)B * h->cfg.latent_channels * N * sizeof(float);
     const size_t out_bytes = (size_t)B * h->hop * N * sizeof(float);
     CK_CUDA(cudaMemcpyAsync(h->lat_io, latents_host, in_bytes, cudaMemcpyHostToDevice, s), "latents upload");
-    mh3a_status st = run_decode(h, h->lat_io, B, N, h->wav_io, s);
+    mh3a_status st = decode_dispatch(h, h->lat_io, B, N, h->wav_io, s);
     if (st) return st;
     CK_CUDA(cudaMemcpyAsync(out_host, h->wav_io, out_bytes, cudaMemcpyDeviceToHost, s), "waveform download");
     CK_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
