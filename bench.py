@@ -295,7 +295,7 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
     if not args.no_graph:
-        dec.set_graph_mode(True)   # the first warm-up decode captures, the rest replay
+        dec.set_graph_mode(True)   # the second warm-up decode captures, later ones replay
     audio_s = B * N / 40.0
     n_stages = len(arch.rates)
 

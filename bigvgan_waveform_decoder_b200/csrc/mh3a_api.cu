@@ -159,6 +159,10 @@ struct mh3a_handle {
     static constexpr int kGraphSlots = 4;
     bool graph_mode = false;
     GraphEntry graphs[kGraphSlots];
+    // keys decoded once without a graph: a key is captured on its second use, so callers that
+    // pass fresh buffers every time never pay for a capture
+    static constexpr int kSeenSlots = 8;
+    GraphEntry seen[kSeenSlots];
     unsigned long long graph_tick = 0;
 };
 
@@ -967,6 +971,26 @@ mh3a_status decode_dispatch(mh3a_handle* h, const float* in, int B, int N, float
     for (auto& g : h->graphs)
         if (g.exec && g.B == B && g.N == N && g.in == in && g.out == out) e = &g;
     if (!e) {
+        // first use of this key: remember it and launch directly
+        mh3a_handle::GraphEntry* k = nullptr;
+        for (auto& g : h->seen)
+            if (g.used && g.B == B && g.N == N && g.in == in && g.out == out) k = &g;
+        if (!k) {
+            k = &h->seen[0];
+            for (auto& g : h->seen) {
+                if (!g.used) { k = &g; break; }
+                if (g.used < k->used) k = &g;
+            }
+            k->B = B;
+            k->N = N;
+            k->in = in;
+            k->out = out;
+            k->used = ++h->graph_tick;
+            return run_decode(h, in, B, N, out, s);
+        }
+        *k = mh3a_handle::GraphEntry{};   // second use: captured below
+    }
+    if (!e) {
         // a free slot, else the least recently used one
         e = &h->graphs[0];
         for (auto& g : h->graphs) {
@@ -1019,6 +1043,7 @@ mh3a_status mh3a_set_graph_mode(mh3a_handle* h, int enable) {
             }
             g = mh3a_handle::GraphEntry{};
         }
+        for (auto& g : h->seen) g = mh3a_handle::GraphEntry{};
     }
     h->graph_mode = enable != 0;
     return MH3A_OK;

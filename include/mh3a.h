@@ -201,16 +201,17 @@ MH3A_API mh3a_status mh3a_amp_stage(mh3a_handle* h, const float* x, int B, int L
 MH3A_API mh3a_status mh3a_amp_stage_static(mh3a_handle* h, const float* x, int B, int L, int stage,
                                            float* out, void* stream);
 
-/* Graph replay of decodes.  With graph mode on, the first mh3a_decode (or mh3a_decode_host)
+/* Graph replay of decodes.  With graph mode on, the second mh3a_decode (or mh3a_decode_host)
  * for a given (B, N, latents pointer, output pointer) captures the decode's kernel launches on
  * the caller's stream into a CUDA graph and instantiates it; that call and every later one with
- * the same four values launch the instantiated graph, which performs exactly the launches of a
- * direct decode (identical results; mh3a_launch_count grows by the same amount) with less launch
- * overhead.  The graph holds the two pointers, so refilling the same input buffer and calling
- * again is the intended use.  Up to 4 graphs are kept per handle (the least recently used one
- * is replaced, after a device synchronisation).  Decodes on the legacy default stream (NULL)
- * or the per-thread default stream, on a stream the caller is capturing, or with
- * mh3a_set_profiling / mh3a_set_kernel_profiling active run their launches directly.
+ * the same four values launch the instantiated graph.  The first call for a key launches
+ * directly, so a caller that passes new buffers every time never pays for a capture.  A replay
+ * performs exactly the launches of a direct decode (identical results; mh3a_launch_count grows
+ * by the same amount) with less launch overhead.  The graph holds the two pointers: refilling
+ * the same input buffer and calling again is the intended use.  Up to 4 graphs are kept per
+ * handle (the least recently used one is replaced, after a device synchronisation).  Decodes
+ * on the legacy default stream (NULL) or the per-thread default stream, on a stream the caller
+ * is capturing, or with mh3a_set_profiling / mh3a_set_kernel_profiling active launch directly.
  * Disabling (enable = 0) synchronises the device and releases every graph.  Capture or
  * instantiation errors return MH3A_ERR_CUDA (mh3a_last_error says which) and leave the stream
  * usable.  Default: off. */
