@@ -22,7 +22,8 @@ MAX_STAGES, MAX_RESBLOCKS, MAX_DILATIONS = 8, 4, 4
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "shape mismatch",
           4: "missing weight", 5: "allocation failed", 6: "CUDA error", 7: "unsupported request"}
 
-EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_create_with_allocator", "mh3a_decode",
+EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_create_with_allocator", "mh3a_create_from_safetensors",
+           "mh3a_decode",
            "mh3a_decode_host",
            "mh3a_amp_stage", "mh3a_set_graph_mode", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
            "mh3a_device_bytes", "mh3a_destroy", "mh3a_status_string", "mh3a_last_error",
@@ -98,6 +99,9 @@ def load():
     L.mh3a_create_with_allocator.argtypes = [C.POINTER(mh3a_config), C.POINTER(mh3a_tensor), C.c_int,
                                              C.POINTER(mh3a_allocator), C.POINTER(vp)]
     L.mh3a_create_with_allocator.restype = C.c_int
+    L.mh3a_create_from_safetensors.argtypes = [C.POINTER(mh3a_config), C.c_char_p, C.POINTER(mh3a_allocator),
+                                               C.POINTER(vp)]
+    L.mh3a_create_from_safetensors.restype = C.c_int
     L.mh3a_decode.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
     L.mh3a_decode.restype = C.c_int
     L.mh3a_decode_host.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
@@ -201,29 +205,37 @@ def _stream_ptr(stream) -> int:
 class Decoder:
     """Owns one mh3a handle on the current CUDA device."""
 
-    def __init__(self, arch, weights: dict, precision: int = MH3A_BF16X3, max_batch: int = 2,
+    def __init__(self, arch, weights, precision: int = MH3A_BF16X3, max_batch: int = 2,
                  max_frames: int = 400, no_clamp: bool = False, allocator=None):
-        """allocator: optional (alloc(bytes) -> int device pointer or 0, release(ptr)) pair that
-        provides the handle's device memory (mh3a_create_with_allocator); it is kept alive with
-        the handle."""
+        """weights: a dict name -> array (mh3a_create), or the path of a safetensors checkpoint
+        (mh3a_create_from_safetensors).  allocator: optional (alloc(bytes) -> int device pointer
+        or 0, release(ptr)) pair that provides the handle's device memory
+        (mh3a_create_with_allocator); it is kept alive with the handle."""
         L = load()
         self.arch = arch
         self.hop = int(np.prod(arch.rates))
         self.latent_channels = arch.latent_channels
         cfg, keep = make_config(arch, precision, max_batch, max_frames, no_clamp)
-        tab, keep2 = make_table(weights)
         h = C.c_void_p()
         self._alloc = None
-        if allocator is None:
-            _check(L.mh3a_create(C.byref(cfg), tab, len(weights), C.byref(h)), "mh3a_create")
-        else:
+        if allocator is not None:
             alloc_py, release_py = allocator
             self._alloc = mh3a_allocator(ALLOC_FN(lambda n, user: alloc_py(int(n)) or None),
                                          RELEASE_FN(lambda ptr, user: release_py(int(ptr))), None)
-            _check(L.mh3a_create_with_allocator(C.byref(cfg), tab, len(weights), C.byref(self._alloc),
-                                                C.byref(h)), "mh3a_create_with_allocator")
+        if isinstance(weights, (str, os.PathLike)):
+            a = C.byref(self._alloc) if self._alloc is not None else None
+            _check(L.mh3a_create_from_safetensors(C.byref(cfg), os.fsencode(weights), a, C.byref(h)),
+                   "mh3a_create_from_safetensors")
+        else:
+            tab, keep2 = make_table(weights)
+            if self._alloc is None:
+                _check(L.mh3a_create(C.byref(cfg), tab, len(weights), C.byref(h)), "mh3a_create")
+            else:
+                _check(L.mh3a_create_with_allocator(C.byref(cfg), tab, len(weights), C.byref(self._alloc),
+                                                    C.byref(h)), "mh3a_create_with_allocator")
+            del keep2
         self._h = h
-        del keep, keep2
+        del keep
 
     @property
     def handle(self):

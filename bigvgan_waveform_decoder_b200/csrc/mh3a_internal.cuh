@@ -3,11 +3,15 @@
 
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <string>
 #include <utility>
 
 #include "mh3a.h"  // include/ is on the include path
 
 namespace mh3a {
+
+// Text returned by mh3a_last_error() on the calling host thread.
+void set_last_error(const std::string& what);
 
 constexpr int kFilterTaps = 12;  // activation filter length (ratio 2: 6 * ratio)
 

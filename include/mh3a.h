@@ -152,6 +152,30 @@ MH3A_API mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh
                                                 int n_weights, const mh3a_allocator* allocator,
                                                 mh3a_handle** out);
 
+/* Build a decoder from the audio VAE component's checkpoint file, the single safetensors file
+ * the FastVideo "minimax_h3_audio_vae" page loads (`mlx_h3_audio_vae_from_dir`,
+ * `mlx_h3_audio_vae_from_file`: `diffusion_pytorch_model.safetensors`).  `path` is a host
+ * NUL-terminated file name.  Format: an 8-byte little-endian header length n, a JSON header of n
+ * bytes mapping tensor names to {"dtype", "shape", "data_offsets": [begin, end]} (plus an
+ * optional "__metadata__" object), then the data section.  Of the file, only tensors named
+ * "dec_in_proj.*" and "decoder.*" (the decode path) are read; every other entry (the encoder's,
+ * the latent statistics' projections) is parsed and skipped.  Those tensors must be stored as
+ * "F32" (the page requires fp32 storage) with 1 to 3 dimensions; "dec_in_proj.weight",
+ * "decoder.conv_pre.weight_v" and "decoder.conv_post.weight_v" must be present (the page's
+ * required decode keys).  The released activation filter buffers ("*.upsample.filter",
+ * "*.downsample.lowpass.filter") are not read: the library builds the same Kaiser-sinc filter.
+ * The tensors are then passed, under their file names, to mh3a_create_with_allocator
+ * (`allocator` may be NULL: cudaMalloc), whose checks apply unchanged.  The file is read with
+ * host buffers that are released before the call returns.
+ * Errors: MH3A_ERR_INVALID_ARG (NULL cfg/path/out; the file cannot be opened or read; a header
+ * length out of range; malformed header JSON; data offsets outside the data section or
+ * disagreeing with the shape), MH3A_ERR_UNSUPPORTED (a decode tensor not stored as F32, or with
+ * more than 3 dimensions), MH3A_ERR_MISSING_WEIGHT (a required key absent; others as reported by
+ * mh3a_create), MH3A_ERR_ALLOC (a host buffer), and every error of mh3a_create.  The reason is in
+ * mh3a_last_error().  On error *out is set to NULL. */
+MH3A_API mh3a_status mh3a_create_from_safetensors(const mh3a_config* cfg, const char* path,
+                                                  const mh3a_allocator* allocator, mh3a_handle** out);
+
 /* Decode latents (device, [B, latent_channels, N]) into a waveform (device, [B, 1, hop*N]),
  * clamped to [-1, 1] unless MH3A_FLAG_NO_CLAMP was configured.  `out` must not overlap
  * `latents`.  1 <= B <= max_batch, 1 <= N <= max_frames, else MH3A_ERR_SHAPE. */
