@@ -22,7 +22,7 @@ MAX_STAGES, MAX_RESBLOCKS, MAX_DILATIONS = 8, 4, 4
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "shape mismatch",
           4: "missing weight", 5: "allocation failed", 6: "CUDA error", 7: "unsupported request"}
 
-EXPORTS = ("mh3a_default_config", "mh3a_create", "mh3a_create_with_allocator", "mh3a_create_from_safetensors",
+EXPORTS = ("mh3a_default_config", "mh3a_config_from_json", "mh3a_create", "mh3a_create_with_allocator", "mh3a_create_from_safetensors",
            "mh3a_decode",
            "mh3a_decode_host",
            "mh3a_amp_stage", "mh3a_set_graph_mode", "mh3a_set_profiling", "mh3a_segment_times", "mh3a_launch_count",
@@ -102,6 +102,9 @@ def load():
     L.mh3a_create_from_safetensors.argtypes = [C.POINTER(mh3a_config), C.c_char_p, C.POINTER(mh3a_allocator),
                                                C.POINTER(vp)]
     L.mh3a_create_from_safetensors.restype = C.c_int
+    L.mh3a_config_from_json.argtypes = [C.c_char_p, C.POINTER(mh3a_config), C.POINTER(C.c_float),
+                                        C.POINTER(C.c_float), C.c_int]
+    L.mh3a_config_from_json.restype = C.c_int
     L.mh3a_decode.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
     L.mh3a_decode.restype = C.c_int
     L.mh3a_decode_host.argtypes = [vp, vp, C.c_int, C.c_int, vp, vp]
@@ -180,6 +183,38 @@ def make_config(arch, precision: int = MH3A_BF16X3, max_batch: int = 2, max_fram
     return cfg, keep
 
 
+class ComponentArch:
+    """The architecture fields make_config reads, from a component's config.json."""
+
+    def __init__(self, cfg: "mh3a_config", mean, std):
+        n = cfg.n_stages
+        self.latent_channels = cfg.latent_channels
+        self.latent_dim = cfg.latent_dim
+        self.decoder_dim = cfg.decoder_dim
+        self.rates = tuple(cfg.rates[i] for i in range(n))
+        self.kernels = tuple(cfg.kernels[i] for i in range(n))
+        self.rb_kernels = tuple(cfg.rb_kernels[j] for j in range(cfg.n_resblocks))
+        self.rb_dilations = tuple(tuple(cfg.rb_dilations[j][m] for m in range(cfg.n_dilations))
+                                  for j in range(cfg.n_resblocks))
+        self.sampling_rate = cfg.sampling_rate
+        self.latents_mean = mean
+        self.latents_std = std
+
+
+def load_config(path) -> ComponentArch:
+    """mh3a_config_from_json: the architecture (and latent statistics) of a config.json."""
+    cfg = mh3a_config()
+    cap = 4096
+    mean = np.zeros(cap, np.float32)
+    std = np.zeros(cap, np.float32)
+    fp = C.POINTER(C.c_float)
+    _check(load().mh3a_config_from_json(os.fsencode(path), C.byref(cfg), mean.ctypes.data_as(fp),
+                                        std.ctypes.data_as(fp), cap), "mh3a_config_from_json")
+    n = cfg.latent_channels
+    return ComponentArch(cfg, mean[:n].copy() if cfg.latents_mean else None,
+                         std[:n].copy() if cfg.latents_std else None)
+
+
 def make_table(weights: dict):
     keep = []
     arr = (mh3a_tensor * len(weights))()
@@ -236,6 +271,25 @@ class Decoder:
             del keep2
         self._h = h
         del keep
+
+    @classmethod
+    def from_component_dir(cls, component_dir, **kw):
+        """The released audio VAE component directory: config.json (mh3a_config_from_json; the
+        defaults when absent) and diffusion_pytorch_model.safetensors
+        (mh3a_create_from_safetensors), as the MLX page's `mlx_h3_audio_vae_from_dir` loads
+        it."""
+        d = os.fspath(component_dir)
+        weights = os.path.join(d, "diffusion_pytorch_model.safetensors")
+        if not os.path.exists(weights):
+            raise FileNotFoundError(f"No audio VAE safetensors under {d}")
+        conf = os.path.join(d, "config.json")
+        if os.path.exists(conf):
+            arch = load_config(conf)
+        else:
+            cfg = mh3a_config()
+            load().mh3a_default_config(C.byref(cfg))
+            arch = ComponentArch(cfg, None, None)
+        return cls(arch, weights, **kw)
 
     @property
     def handle(self):

@@ -114,6 +114,27 @@ typedef struct mh3a_handle mh3a_handle;
  * statistics, max_batch 2, max_frames 400. */
 MH3A_API void mh3a_default_config(mh3a_config* cfg);
 
+/* Fill *cfg from a released component's config.json: the diffusers
+ * "AutoencoderKLMiniMaxH3Audio" constructor arguments, which the FastVideo
+ * "minimax_h3_audio_vae" page's `MiniMaxH3AudioVAEConfigView.from_vae_dir` reads from the
+ * component directory.  Starts from mh3a_default_config and takes latent_channels, latent_dim,
+ * decoder_dim, decoder_rates, decoder_kernel_sizes, resblock_kernel_sizes,
+ * resblock_dilation_sizes, sampling_rate and latents_mean / latents_std (null or a list of
+ * latent_channels numbers); every other key is skipped.  A list that changes a count
+ * (decoder_rates, resblock_kernel_sizes) needs its companion list (decoder_kernel_sizes,
+ * resblock_dilation_sizes).  Statistics are written to the caller's host arrays latents_mean /
+ * latents_std (cap floats each; NULL is allowed when the file has none) and cfg->latents_mean /
+ * latents_std point at them, so those arrays must outlive the mh3a_create that uses *cfg.
+ * Precision, flags and workspace limits keep their defaults for the caller to set.  The values
+ * themselves are checked by mh3a_create.
+ * Errors: MH3A_ERR_INVALID_ARG (NULL path/cfg, negative cap, unreadable file, malformed JSON,
+ * a field of the wrong type), MH3A_ERR_CONFIG (more stages, blocks or dilations than the MAX_*
+ * limits; list lengths that disagree), MH3A_ERR_SHAPE (a statistics list not of latent_channels
+ * values, or no caller array large enough).  The reason is in mh3a_last_error(); on error *cfg
+ * is left unchanged. */
+MH3A_API mh3a_status mh3a_config_from_json(const char* path, mh3a_config* cfg, float* latents_mean,
+                                           float* latents_std, int cap);
+
 /* Build a decoder on the current CUDA device.  Copies the weight table to device memory,
  * folds every weight norm w = g * v / ||v|| (MLX page `_wn_weight`) and the optional latent
  * denormalisation into the weights, builds the Kaiser-sinc activation filter (MLX page

@@ -178,3 +178,122 @@ def test_file_handle_decodes_like_the_table_handle(tmp_path):
     finally:
         b.close()
         a.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# config.json (mh3a_config_from_json, binding.load_config, Decoder.from_component_dir)
+# ---------------------------------------------------------------------------------------------
+
+def _released_like_config(**over):
+    """The diffusers constructor arguments with their defaults (the pages say these mirror the
+    released audio_vae/config.json), plus diffusers' bookkeeping keys."""
+    c = {"_class_name": "AutoencoderKLMiniMaxH3Audio", "_diffusers_version": "0.0.0",
+         "encoder_dim": 64, "encoder_rates": [2, 4, 4, 5, 5], "latent_dim": 2048, "latent_channels": 32,
+         "num_attention_heads": 8, "decoder_dim": 1024, "decoder_rates": [5, 5, 2, 2, 2, 2, 2],
+         "decoder_kernel_sizes": [9, 9, 4, 4, 4, 4, 4], "resblock_kernel_sizes": [3, 7, 11],
+         "resblock_dilation_sizes": [[1, 3, 5], [1, 3, 5], [1, 3, 5]], "sampling_rate": 32000,
+         "latents_mean": None, "latents_std": None}
+    c.update(over)
+    return c
+
+
+def _cfg_status(path, cap=64, with_buffers=True):
+    cfg = Bd.mh3a_config()
+    m = np.zeros(max(cap, 1), np.float32)
+    s = np.zeros(max(cap, 1), np.float32)
+    fp = C.POINTER(C.c_float)
+    st = Bd.load().mh3a_config_from_json(str(path).encode(), C.byref(cfg),
+                                         m.ctypes.data_as(fp) if with_buffers else None,
+                                         s.ctypes.data_as(fp) if with_buffers else None, cap)
+    return st, cfg, m, s, Bd.load().mh3a_last_error().decode()
+
+
+def test_released_like_config_gives_the_defaults(tmp_path):
+    p = tmp_path / "config.json"
+    p.write_text(json.dumps(_released_like_config()))
+    a = Bd.load_config(p)
+    d = S.Arch()
+    assert (a.latent_channels, a.latent_dim, a.decoder_dim) == (d.latent_channels, d.latent_dim, d.decoder_dim)
+    assert a.rates == tuple(d.rates) and a.kernels == tuple(d.kernels)
+    assert a.rb_kernels == tuple(d.rb_kernels) and a.rb_dilations == tuple(tuple(r) for r in d.rb_dilations)
+    assert a.sampling_rate == 32000 and a.latents_mean is None and a.latents_std is None
+
+
+def test_config_with_statistics_and_a_smaller_architecture(tmp_path):
+    rng = np.random.default_rng(3)
+    mean = rng.uniform(-0.5, 0.5, 4).tolist()
+    std = rng.uniform(0.5, 1.5, 4).tolist()
+    p = tmp_path / "config.json"
+    p.write_text(json.dumps(_released_like_config(
+        latent_channels=4, latent_dim=32, decoder_dim=128, decoder_rates=[8, 5, 4, 5],
+        decoder_kernel_sizes=[16, 11, 8, 11], resblock_kernel_sizes=[3, 5],
+        resblock_dilation_sizes=[[1, 2], [1, 3]], latents_mean=mean, latents_std=std)))
+    a = Bd.load_config(p)
+    assert a.latent_channels == 4 and a.rates == (8, 5, 4, 5) and a.kernels == (16, 11, 8, 11)
+    assert a.rb_kernels == (3, 5) and a.rb_dilations == ((1, 2), (1, 3))
+    np.testing.assert_array_equal(a.latents_mean, np.float32(mean))
+    np.testing.assert_array_equal(a.latents_std, np.float32(std))
+
+
+@pytest.mark.parametrize("case,expect", [
+    ({"decoder_rates": [5, 5, 2, 2, 2, 16]}, 2),                                 # stage count, no kernels
+    ({"decoder_kernel_sizes": [9, 9, 4]}, 2),                                    # 3 kernels, 7 stages
+    ({"decoder_rates": [2] * 9, "decoder_kernel_sizes": [4] * 9}, 2),            # beyond MAX_STAGES
+    ({"resblock_dilation_sizes": [[1, 3, 5], [1, 3]]}, 2),                       # 2 rows for 3 blocks
+    ({"resblock_dilation_sizes": [[1, 3, 5], [1, 3], [1, 5, 7]]}, 2),            # ragged rows
+    ({"resblock_kernel_sizes": [3, 7]}, 2),                                      # block count, no dilations
+    ({"latents_mean": [0.0] * 31}, 3),                                           # 31 values for 32 channels
+    ({"latent_dim": -2048}, 1),
+    ({"latent_channels": 32.5}, 1),
+    ({"decoder_rates": "5,5,2"}, 1),
+])
+def test_bad_configs_are_rejected(tmp_path, case, expect):
+    p = tmp_path / "config.json"
+    p.write_text(json.dumps(_released_like_config(**case)))
+    st, cfg, m, s, err = _cfg_status(p)
+    assert st == expect, (case, st, err)
+    assert err
+
+
+def test_malformed_config_and_small_buffers(tmp_path):
+    p = tmp_path / "config.json"
+    p.write_text('{"latent_dim": 2048,')
+    assert _cfg_status(p)[0] == 1
+    p.write_text(json.dumps(_released_like_config(latents_mean=[0.1] * 32)))
+    assert _cfg_status(p, cap=16)[0] == 3                      # 32 values, room for 16
+    assert _cfg_status(p, cap=64, with_buffers=False)[0] == 3   # statistics but no buffers
+    st, cfg, m, s, err = _cfg_status(p, cap=64)
+    assert st == 0 and bool(cfg.latents_mean) and not bool(cfg.latents_std)
+    np.testing.assert_array_equal(m[:32], np.float32([0.1] * 32))
+    assert _cfg_status(tmp_path / "nothing.json")[0] == 1
+
+
+def test_component_dir_needs_the_weights_file(tmp_path):
+    (tmp_path / "config.json").write_text(json.dumps(_released_like_config()))
+    with pytest.raises(FileNotFoundError):
+        Bd.Decoder.from_component_dir(tmp_path)
+
+
+@pytest.mark.gpu
+def test_component_dir_decodes_like_the_table_handle(tmp_path):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    rng = np.random.default_rng(9)
+    mean = rng.uniform(-0.5, 0.5, 32).astype(np.float32)
+    std = rng.uniform(0.5, 1.5, 32).astype(np.float32)
+    arch = S.Arch(latents_mean=mean, latents_std=std)
+    w = S.workload_weights(0, S.Arch())
+    (tmp_path / "config.json").write_text(json.dumps(_released_like_config(
+        latents_mean=mean.tolist(), latents_std=std.tolist())))
+    write_st(tmp_path / "diffusion_pytorch_model.safetensors", w, metadata={"format": "pt"})
+    z = torch.from_numpy(S.make_latents(2, 8, 32, 78)).cuda()
+    a = Bd.Decoder(arch, w, max_batch=2, max_frames=8)
+    b = Bd.Decoder.from_component_dir(tmp_path, max_batch=2, max_frames=8)
+    try:
+        assert torch.equal(a.decode(z), b.decode(z))
+        b.check_device_error()
+    finally:
+        b.close()
+        a.close()
