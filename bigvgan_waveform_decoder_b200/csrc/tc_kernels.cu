@@ -1062,7 +1062,13 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
                     return -1;
     }
     constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * (convt_grouped(R) ? R * NT : NT) * 16;
-    p.tpu = std::max(1, std::min(kumax, 16384 / TAPB));   // weight copies of about 16 KB
+    // Weight copies of about 16 KB; the AMP convs of 32 to 128 channels take up to 64 KB per
+    // copy, which halves or quarters the ring's per-copy commits and waits (measured per launch:
+    // 128 channels 82 -> 77 us, 64 channels 58 -> 55 us, 32 channels 51 -> 49 us; the widest
+    // tiles and the narrow 2-group chunks stay at 16 KB, where larger copies measured slower or
+    // equal).
+    const int wbytes = (R == 1 && KGT == 4 && NT <= 128) ? 65536 : 16384;
+    p.tpu = std::max(1, std::min(kumax, wbytes / TAPB));
     PsSched sc{};
     sc.n_ot = (p.Cout + NT - 1) / NT;
     sc.per_job = p.B * p.tiles_t * sc.n_ot;
