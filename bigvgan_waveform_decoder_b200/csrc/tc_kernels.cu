@@ -18,7 +18,7 @@
 //
 // Accumulation: the tensor core rounds its fp32 accumulator toward zero at every instruction,
 // so a long K loop into one accumulator builds a bias of about (instructions) x 2^-24
-// relative.  k_gemm_ps bounds every accumulator to one pass of at most 8 K-steps and adds the
+// relative.  k_gemm_ps bounds every accumulator to one pass of at most 16 K-steps and adds the
 // passes in fp32 registers with round-to-nearest; k_conv_tc gives each M tile NACC
 // accumulators (head x head products rotating over the first NACC-1 by chunk, the cross terms
 // in the last) and adds them in the epilogue.
@@ -461,10 +461,10 @@ struct GemmParams {
 
 // ----------------------------------------------------------------------------------------------
 // persistent AMP GEMM: one CTA per SM walks a list of output tiles (job, item, 128 MT time rows,
-// NT output channels).  The tile's K loop is cut into passes of at most 8 MMA K-steps; each
+// NT output channels).  The tile's K loop is cut into passes of at most 16 MMA K-steps; each
 // pass accumulates head x head and both cross products into one of two TMEM buffers, and the
 // epilogue warps fold the finished buffer into fp32 registers (round to nearest) while the
-// tensor core fills the other.  A pass therefore holds at most 24 truncating accumulations,
+// tensor core fills the other.  A pass therefore holds at most 48 truncating accumulations,
 // the epilogue of one tile overlaps the MMAs of the next, and A / B stream through rings of
 // bulk copies that run several stages ahead.
 // ----------------------------------------------------------------------------------------------
@@ -1073,8 +1073,11 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     sc.n_ot = (p.Cout + NT - 1) / NT;
     sc.per_job = p.B * p.tiles_t * sc.n_ot;
     sc.ntiles = njobs * sc.per_job;
-    // passes of 8 MMA K-steps; the upsampler's pass is one whole chunk
-    sc.pu = (R > 1) ? 64 : (KGT == 4) ? 4 : 8;
+    // Passes of 8 MMA K-steps (4 taps of 32 channels) at the widest tiles; 16 K-steps (8 taps)
+    // for the 32- to 128-channel convs and 16 taps of the 16-channel chunks, where fewer
+    // accumulator drains measured 1-3 us per launch faster; the upsampler's pass is one whole
+    // chunk.  A pass holds at most 48 truncating accumulations per accumulator column.
+    sc.pu = (R > 1) ? 64 : (KGT == 4) ? ((NT <= 128) ? 8 : 4) : 16;
     PsPlan pl{};
     pl.RS = 128 * MT + span;
     pl.SA = 2 * KGT * pl.RS * 16;
