@@ -1062,12 +1062,13 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
                     return -1;
     }
     constexpr int TAPB = 2 * (KGT == 1 ? 2 : KGT) * (convt_grouped(R) ? R * NT : NT) * 16;
-    // Weight copies of about 16 KB; the AMP convs of 32 to 128 channels take up to 64 KB per
-    // copy, which halves or quarters the ring's per-copy commits and waits (measured per launch:
-    // 128 channels 82 -> 77 us, 64 channels 58 -> 55 us, 32 channels 51 -> 49 us; the widest
-    // tiles and the narrow 2-group chunks stay at 16 KB, where larger copies measured slower or
-    // equal).
-    const int wbytes = (R == 1 && KGT == 4 && NT <= 128) ? 65536 : 16384;
+    // Weight copies of about 16 KB; the AMP convs of 32 to 128 channels and the upsamplers take
+    // up to 64 KB per copy, which halves or quarters the ring's per-copy commits and waits
+    // (measured per launch: 128 channels 82 -> 77 us, 64 channels 58 -> 55 us, 32 channels
+    // 51 -> 49 us; upsamplers 1024 -> 512 channels 66.5 -> 60.5 us, 512 -> 256 70.7 -> 64.5 us,
+    // 256 -> 128 60.4 -> 58.3 us; 32 KB copies gained only the last).  The widest AMP tiles and
+    // the narrow 2-group chunks stay at 16 KB, where larger copies measured slower or equal.
+    const int wbytes = (R > 1 || (KGT == 4 && NT <= 128)) ? 65536 : 16384;
     p.tpu = std::max(1, std::min(kumax, wbytes / TAPB));
     PsSched sc{};
     sc.n_ot = (p.Cout + NT - 1) / NT;
