@@ -151,20 +151,22 @@ __global__ void __launch_bounds__(NT_ACT, 4) k_act_split(const ActParams p) {
     }
 }
 
-// Input value of channel row `ci` (index into [B, C, L]) in the form the split takes.
+// Input value of channel row `ci` (index into [B, C, L]) in the form the split takes.  The
+// inputs (conv_pre's partial outputs, a stage's block outputs) are read here for the last time,
+// so the loads are streaming (evict-first): measured 5 us less per decode over the seven splits.
 __device__ __forceinline__ float split_in(const SplitParams& p, long long ci) {
-    if (p.x3) return ((__ldg(p.x0 + ci) + __ldg(p.x1 + ci)) + __ldg(p.x2 + ci)) + __ldg(p.x3 + ci);
-    if (p.x1) return (__ldg(p.x0 + ci) + __ldg(p.x1 + ci) + __ldg(p.x2 + ci)) * (1.0f / 3.0f);
-    return __ldg(p.x0 + ci);
+    if (p.x3) return ((__ldcs(p.x0 + ci) + __ldcs(p.x1 + ci)) + __ldcs(p.x2 + ci)) + __ldcs(p.x3 + ci);
+    if (p.x1) return (__ldcs(p.x0 + ci) + __ldcs(p.x1 + ci) + __ldcs(p.x2 + ci)) * (1.0f / 3.0f);
+    return __ldcs(p.x0 + ci);
 }
 
 __device__ __forceinline__ float2 split_in2(const SplitParams& p, long long ci) {
-    const float2 a = __ldg(reinterpret_cast<const float2*>(p.x0 + ci));
+    const float2 a = __ldcs(reinterpret_cast<const float2*>(p.x0 + ci));
     if (!p.x1) return a;
-    const float2 b = __ldg(reinterpret_cast<const float2*>(p.x1 + ci));
-    const float2 c = __ldg(reinterpret_cast<const float2*>(p.x2 + ci));
+    const float2 b = __ldcs(reinterpret_cast<const float2*>(p.x1 + ci));
+    const float2 c = __ldcs(reinterpret_cast<const float2*>(p.x2 + ci));
     if (p.x3) {
-        const float2 d = __ldg(reinterpret_cast<const float2*>(p.x3 + ci));
+        const float2 d = __ldcs(reinterpret_cast<const float2*>(p.x3 + ci));
         return make_float2(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y);
     }
     return make_float2((a.x + b.x + c.x) * (1.0f / 3.0f), (a.y + b.y + c.y) * (1.0f / 3.0f));
@@ -266,13 +268,21 @@ __global__ void __launch_bounds__(NT_ACT) k_proj_split(const ProjSplitParams p) 
 // grid: x = output tiles of TT - (K - 1) samples, y = B.  Warp c stages the mean input window of
 // channel c, forms its 512 activation values of rows [t0 - pad, t0 - pad + 512) with the same
 // lane routine as k_act_split, and parks them in shared memory (zero outside [0, L): the conv's
-// padding); then every thread forms up to two outputs from the 8 x K window.
+// padding); then every thread forms up to two outputs from the 8 x K window.  The three block
+// outputs' windows arrive as asynchronous copies, all in flight at once (a load loop waited for
+// each round of loads: 41 -> 35 us per launch at B = 2, L = 320000); blocks 1 and 2 land in a
+// staging area that the activation rows reuse afterwards.
+constexpr int POST_STAGE = 2 * 8 * XF;   // floats: the windows of blocks 1 and 2, unskewed
+static_assert(POST_STAGE >= 8 * TT, "the activation rows fit in the staging area");
+constexpr int POST_SMEM = (8 * XF_P + POST_STAGE + 8 * kPostMaxK) * 4;   // bytes (dynamic)
 __global__ void __launch_bounds__(NT_ACT) k_post_act(const PostParams p) {
     ptx::grid_dep_wait();     // launched as a programmatic dependent (see launch_dependent)
     ptx::grid_dep_launch();
-    __shared__ __align__(16) float xsb[8 * XF_P];
-    __shared__ __align__(16) float arow[8][TT];
-    __shared__ float wsh[8 * kPostMaxK];
+    extern __shared__ __align__(16) float post_smem[];
+    float* xsb = post_smem;                          // [8][XF_P] skewed mean windows
+    float* stage = xsb + 8 * XF_P;                   // [2][8][XF], then [8][TT] activation rows
+    float* wsh = stage + POST_STAGE;                 // [8 * K] conv_post weights
+    float (*arow)[TT] = reinterpret_cast<float (*)[TT]>(stage);
     const int L = p.L, K = p.K, TO = TT - (K - 1);
     const int b = blockIdx.y;
     const int t0 = blockIdx.x * TO;
@@ -280,14 +290,27 @@ __global__ void __launch_bounds__(NT_ACT) k_post_act(const PostParams p) {
     const int tid = threadIdx.x, c = tid >> 5, lane = tid & 31;
     for (int i = tid; i < 8 * K; i += NT_ACT) wsh[i] = __ldg(p.w + i);
     float* xs = xsb + c * XF_P;
+    float* w1 = stage + c * XF;
+    float* w2 = stage + (8 + c) * XF;
     const long long rb = ((long long)b * 8 + c) * L;
     const bool edge = !(tw >= 8 && tw + TT + 8 <= L);
-    // mean of the three block outputs over x[tw - 8, tw + TT + 8), replicate-clamped at the ends
-    for (int i = lane; i < XF; i += 32) {
-        const long long g = rb + clampi(tw - 8 + i, 0, L - 1);
-        xs[skew(i)] = (__ldg(p.x0 + g) + __ldg(p.x1 + g) + __ldg(p.x2 + g)) / 3.0f;
+    // the three block outputs over x[tw - 8, tw + TT + 8), replicate-clamped at the ends, then
+    // their mean into the skewed window
+#pragma unroll
+    for (int k = 0; k < (XF + 31) / 32; ++k) {
+        const int i = lane + 32 * k;
+        if (i < XF) {
+            const long long g = rb + clampi(tw - 8 + i, 0, L - 1);
+            ptx::cp_async4(xs + skew(i), p.x0 + g);
+            ptx::cp_async4(w1 + i, p.x1 + g);
+            ptx::cp_async4(w2 + i, p.x2 + g);
+        }
     }
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
     __syncwarp();
+    for (int i = lane; i < XF; i += 32) xs[skew(i)] = (xs[skew(i)] + w1[i] + w2[i]) / 3.0f;
+    __syncthreads();   // every warp is done with the staging area before it holds activation rows
     const float al = __ldg(p.alpha + c), ib = __ldg(p.inv_beta + c);
     float a[RUN];
     if (edge) actm::act_lane<RUN, true>(p.filt, xs, al, ib, tw, L, a);
@@ -351,7 +374,9 @@ int launch_post_act(const PostParams& p, cudaStream_t s) {
         return -1;
     const int TO = TT - (p.K - 1);
     dim3 grid((p.L + TO - 1) / TO, p.B);
-    return launch_dependent(k_post_act, grid, dim3(NT_ACT), 0, s, p) == cudaSuccess ? 1 : -1;
+    if (cudaFuncSetAttribute(k_post_act, cudaFuncAttributeMaxDynamicSharedMemorySize, POST_SMEM) != cudaSuccess)
+        return -1;
+    return launch_dependent(k_post_act, grid, dim3(NT_ACT), POST_SMEM, s, p) == cudaSuccess ? 1 : -1;
 }
 
 int launch_proj_split(const ProjSplitParams& p, cudaStream_t s) {
