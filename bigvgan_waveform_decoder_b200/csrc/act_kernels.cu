@@ -349,8 +349,16 @@ __global__ void __launch_bounds__(NT_ACT) k_post_act(const PostParams p) {
                 y0 = (y0 < -1.f) ? -1.f : ((y0 > 1.f) ? 1.f : y0);
                 y1 = (y1 < -1.f) ? -1.f : ((y1 > 1.f) ? 1.f : y1);
             }
-            p.out[(long long)b * L + t0 + q] = y0;
-            if (q + 1 < TO && t0 + q + 1 < L) p.out[(long long)b * L + t0 + q + 1] = y1;
+            // one 8-byte store per pair where aligned (full 256-byte warp stores, which also
+            // suits an output in mapped host memory)
+            float* o = p.out + (long long)b * L + t0 + q;
+            const bool pair = q + 1 < TO && t0 + q + 1 < L;
+            if (pair && (reinterpret_cast<uintptr_t>(o) & 7) == 0) {
+                *reinterpret_cast<float2*>(o) = make_float2(y0, y1);
+            } else {
+                o[0] = y0;
+                if (pair) o[1] = y1;
+            }
         }
     } else {
         for (int q = tid; q < TO; q += NT_ACT) {

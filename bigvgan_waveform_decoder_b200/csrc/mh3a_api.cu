@@ -1062,10 +1062,23 @@ mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, i
     cudaStream_t s = (cudaStream_t)stream;
     const size_t in_bytes = (size_t)B * h->cfg.latent_channels * N * sizeof(float);
     const size_t out_bytes = (size_t)B * h->hop * N * sizeof(float);
+    // A pinned output buffer that the current device can address (page-locked memory from
+    // cudaHostAlloc / cudaMallocHost is mapped into the device's address space under unified
+    // addressing) is written by the decode's last kernel directly: the waveform crosses the bus
+    // while that kernel runs instead of in a copy after it.  Any other host memory gets the
+    // device waveform buffer and a copy.
+    float* out_mapped = nullptr;
+    cudaPointerAttributes pa{};
+    if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess) {
+        if (pa.type == cudaMemoryTypeHost && pa.devicePointer) out_mapped = static_cast<float*>(pa.devicePointer);
+    } else {
+        (void)cudaGetLastError();   // not a pointer the runtime knows: plain host memory
+    }
     CK_CUDA(cudaMemcpyAsync(h->lat_io, latents_host, in_bytes, cudaMemcpyHostToDevice, s), "latents upload");
-    mh3a_status st = decode_dispatch(h, h->lat_io, B, N, h->wav_io, s);
+    mh3a_status st = decode_dispatch(h, h->lat_io, B, N, out_mapped ? out_mapped : h->wav_io, s);
     if (st) return st;
-    CK_CUDA(cudaMemcpyAsync(out_host, h->wav_io, out_bytes, cudaMemcpyDeviceToHost, s), "waveform download");
+    if (!out_mapped)
+        CK_CUDA(cudaMemcpyAsync(out_host, h->wav_io, out_bytes, cudaMemcpyDeviceToHost, s), "waveform download");
     CK_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
     return MH3A_OK;
 }

@@ -203,9 +203,13 @@ MH3A_API mh3a_status mh3a_create_from_safetensors(const mh3a_config* cfg, const 
 MH3A_API mh3a_status mh3a_decode(mh3a_handle* h, const float* latents, int B, int N, float* out,
                         void* stream);
 
-/* The same decode from and to HOST memory: copies the latents in, decodes, copies the
- * waveform out, all on `stream`, and waits for the stream before returning.  Pinned host
- * buffers give the fastest copies.  Same shape limits as mh3a_decode. */
+/* The same decode from and to HOST memory: copies the latents in, decodes, and delivers the
+ * waveform to `out_host`, all on `stream`, and waits for the stream before returning.  When
+ * `out_host` is page-locked memory that the current device can address (cudaHostAlloc /
+ * cudaMallocHost memory, e.g. a pinned torch tensor, under unified addressing), the decode's
+ * last kernel stores the waveform into it directly, so the transfer overlaps that kernel;
+ * other host memory receives a device-to-host copy after the decode.  Pinned host buffers
+ * give the fastest transfers.  Same shape limits as mh3a_decode. */
 MH3A_API mh3a_status mh3a_decode_host(mh3a_handle* h, const float* latents_host, int B, int N,
                              float* out_host, void* stream);
 

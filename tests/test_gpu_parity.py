@@ -154,15 +154,30 @@ def test_batch_independence_and_determinism(dev, full_weights):
         np.testing.assert_array_equal(y1[0], y2[b])
 
 
-def test_decode_host_matches_device(dev, full_weights):
+@pytest.mark.parametrize("prec", [Bd.MH3A_FP32, Bd.MH3A_BF16X3], ids=["FP32", "BF16X3"])
+@pytest.mark.parametrize("out_kind", ["pinned", "pinned_odd_offset", "pageable"])
+def test_decode_host_matches_device(dev, full_weights, prec, out_kind):
+    """Host-buffer decode == device decode bit for bit, whether the waveform reaches host memory
+    through the last kernel's direct stores (pinned output, also 4 bytes off an 8-byte boundary)
+    or through a copy (pageable output)."""
     arch = S.Arch()
     z = S.make_latents(2, 6, 32, 78)
-    d = decoder(arch, full_weights, Bd.MH3A_FP32, max_batch=2, max_frames=64)
+    d = decoder(arch, full_weights, prec, max_batch=2, max_frames=64)
     yd = d.decode(torch.from_numpy(z).to(dev)).cpu().numpy()
     zp = torch.from_numpy(z).pin_memory()
-    yp = torch.empty((2, 1, 800 * 6), dtype=torch.float32).pin_memory()
+    n = 2 * 800 * 6
+    if out_kind == "pinned":
+        yp = torch.full((2, 1, 800 * 6), float("nan"), dtype=torch.float32).pin_memory()
+    elif out_kind == "pinned_odd_offset":
+        big = torch.full((n + 1,), float("nan"), dtype=torch.float32).pin_memory()
+        yp = big[1:].view(2, 1, 800 * 6)
+        assert yp.data_ptr() % 8 == 4
+    else:
+        yp = torch.full((2, 1, 800 * 6), float("nan"), dtype=torch.float32)
     d.decode_host(zp, yp)
     np.testing.assert_array_equal(yp.numpy(), yd)
+    if out_kind == "pinned_odd_offset":
+        assert np.isnan(big[0].item())   # nothing written before the buffer
 
 
 def test_denormalised_decode(dev, full_weights):
