@@ -244,6 +244,19 @@ def extra_amp_stage(Bd, PM, peaks, p_tc, p_fp32, flush, stream, dev, steps: int)
             "l2": "flushed between calls"}
 
 
+PROFILER_ENV = ("NV_NSIGHT_INJECTION_TRANSPORT_TYPE", "NV_COMPUTE_PROFILER_PERFWORKS_DIR",
+                "CUDA_INJECTION64_PATH")
+
+
+def graphs_allowed() -> bool:
+    """False when a profiler has injected itself into the CUDA runtime (Nsight Compute sets the
+    first two variables in the program it starts; CUDA_INJECTION64_PATH is the runtime's own
+    injection hook).  Under ncu, the replay of a captured decode -- kernels chained by
+    programmatic dependent launch -- failed to launch, so a profiled run launches every decode
+    directly: the same kernels, arguments and order."""
+    return not any(os.environ.get(k) for k in PROFILER_ENV)
+
+
 def extra_batched(arch_w, Bd, flush, stream, dev, steps: int) -> dict:
     """The batched 20 s decode: B=16, N=800, per-channel latent denormalisation, seed 4."""
     import torch
@@ -252,7 +265,7 @@ def extra_batched(arch_w, Bd, flush, stream, dev, steps: int) -> dict:
     arch, w, z = arch_w
     B, _, N = z.shape
     dec = Bd.Decoder(arch, w, precision=Bd.MH3A_BF16X3, max_batch=B, max_frames=N)
-    dec.set_graph_mode(True)
+    dec.set_graph_mode(graphs_allowed())
     x = torch.from_numpy(z).to(dev)
     out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
     for _ in range(2):
@@ -287,6 +300,7 @@ def run_ours(args):
     arch, w, _ = S.workload_inputs(WORKLOAD)
     z = S.make_latents(B, N, arch.latent_channels, wl.seed + 1000 * rank)
     precision = Bd.MH3A_BF16X3 if args.precision == "bf16x3" else Bd.MH3A_FP32
+    use_graph = not args.no_graph and graphs_allowed()
     dec = Bd.Decoder(arch, w, precision=precision, max_batch=B, max_frames=N)
     x = torch.from_numpy(z).to(dev)
     out = torch.empty((B, 1, dec.hop * N), device=dev, dtype=torch.float32)
@@ -296,7 +310,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
-    if not args.no_graph:
+    if use_graph:
         dec.set_graph_mode(True)   # the second warm-up decode captures, later ones replay
     audio_s = B * N / 40.0
     n_stages = len(arch.rates)
@@ -419,7 +433,7 @@ def run_ours(args):
         "config": {"workload": f"decode B={B} N={N} (10 s stereo, 2 x 320000 samples) per GPU",
                    "global_batch": B * world, "latent_frames": N, "replicas": world,
                    "weights": "random init, seed 3", "l2": "flushed between steps (256 MiB write)",
-                   "statistic": "median step", "cuda_graph": not args.no_graph},
+                   "statistic": "median step", "cuda_graph": use_graph},
         "roofline": roofline,
         "roofline_activation": roofline_act,
         "e2e": {"value": e2e_value, "unit": UNIT,
