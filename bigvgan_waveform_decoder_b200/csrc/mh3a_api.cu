@@ -41,6 +41,7 @@ constexpr int kMaxSegments = 2 + 2 * MH3A_MAX_STAGES + 1;
 // sequence at least the largest conv padding, after it the largest tile overhang (2 x 128
 // rows) plus that padding.
 constexpr int kApadL = 32;
+constexpr int kMsSlot = 3;   // the A operand pair the fused upsampler input split writes
 constexpr int kApadR = 4 * 128 + 32;
 
 // Kaiser-windowed sinc low-pass of the activation (FastVideo "minimax_h3_audio_vae" page,
@@ -131,6 +132,10 @@ struct mh3a_handle {
     void* A_hi[MH3A_MAX_RESBLOCKS] = {};   // tensor-core A operands (activations, bf16 heads)
     void* A_lo[MH3A_MAX_RESBLOCKS] = {};   //   and tails, with zero padding rows
     long long a_cap = 0;                   // bf16 elements per A array
+    // The fused upsampler input split (three residual blocks): the last AMP layer of a 16- or
+    // 32-channel stage writes the next upsampler's operand into A_hi/A_lo[3] (no operand of that
+    // layer).
+    bool ms_on = false;
     float* lat_io = nullptr;   // host-API staging
     float* wav_io = nullptr;
     int* dev_err = nullptr;    // 64 ints: [0] set by a tensor-core kernel whose bounded wait timed
@@ -339,7 +344,8 @@ mh3a_status counted(mh3a_handle* h, int n) {
 
 // The six residual-chain launches of one AMP stage: input h (B, C, L); the per-block running
 // sums end in h->X[j].  Every launch covers all residual blocks (blockIdx.z).
-mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cudaStream_t s) {
+mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cudaStream_t s,
+                    const MeanSplitTarget* ms = nullptr) {
     const mh3a_config& c = h->cfg;
     const int C = stage_channels(c, stage);
     const int nrb = c.n_resblocks;
@@ -402,7 +408,9 @@ mh3a_status run_amp(mh3a_handle* h, int stage, const float* in, int B, int L, cu
                 if (st) return st;
                 if (kprof) CK_CUDA(cudaEventRecord(h->kev[li][1], s), "cudaEventRecord");
                 const long long Lpad = (long long)L + kApadL + kApadR;
-                n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err, h->dev_err + 16);
+                const bool last = m == c.n_dilations - 1 && half == 1;
+                n = launch_amp_gemm_tc(p, nrb, h->tc[stage], m, half, h->A_hi, h->A_lo, kApadL, Lpad, s, h->dev_err,
+                                       h->dev_err + 16, last ? ms : nullptr);
                 if (kprof && n > 0) {
                     CK_CUDA(cudaEventRecord(h->kev[li][2], s), "cudaEventRecord");
                     if (li == 5) {
@@ -537,6 +545,7 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         if ((st = record(h, s))) return st;
     }
     int C = c.decoder_dim, L = N;
+    bool ms_done = false;
     for (int i = 0; i < c.n_stages; ++i) {
         ConvTParams q{};
         const bool mean3 = (i > 0);
@@ -558,7 +567,11 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
             return MH3A_ERR_UNSUPPORTED;
         }
         int nl;
-        if (i == 0 && h->pre_tc) {
+        if (i > 0 && ms_done) {
+            // the previous stage's last layer wrote this upsampler's operand rows
+            nl = launch_convT_gemm(q, h->tc[i], h->A_hi[kMsSlot], h->A_lo[kMsSlot], kApadL,
+                                   (long long)L + kApadL + kApadR, s, h->dev_err, h->dev_err + 16);
+        } else if (i == 0 && h->pre_tc) {
             // conv_pre left its output as partial sums over input-channel slices
             float* const* part = pre_parts(h);
             if (!h->ups_tc[i]) return MH3A_ERR_UNSUPPORTED;
@@ -576,7 +589,11 @@ mh3a_status run_decode(mh3a_handle* h, const float* lat, int B, int N, float* ou
         if ((st = record(h, s))) return st;
         C /= 2;
         L *= c.rates[i];
-        if ((st = run_amp(h, i, h->H, B, L, s))) return st;
+        // the stage's last layer also forms the next upsampler's operand where it can
+        ms_done = h->ms_on && i + 1 < c.n_stages && h->stage_tc[i] && !h->stage_fused[i] && h->ups_tc[i + 1] &&
+                  amp_gemm_split_fusable(C) && (long long)B * C * ((long long)L + kApadL + kApadR) <= h->a_cap;
+        MeanSplitTarget mst{h->A_hi[kMsSlot], h->A_lo[kMsSlot], kApadL, (long long)L + kApadL + kApadR};
+        if ((st = run_amp(h, i, h->H, B, L, s, ms_done ? &mst : nullptr))) return st;
         if ((st = record(h, s))) return st;
     }
     // activation_post + conv_post + clamp, reading the mean of the last stage's blocks
@@ -916,7 +933,19 @@ mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh3a_tensor
         h->a_cap = need * c.max_batch;
     }
     const long long n_a = rnd((h->a_cap + 1) / 2);   // floats per head or tail array
-    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64 + 2 * c.n_resblocks * n_a;
+    // the fused upsampler input split writes a fourth operand pair
+    h->ms_on = c.n_resblocks == 3 && n_a > 0;
+    if (h->ms_on) {
+        bool any = false;
+        int Cs = c.decoder_dim;
+        for (int i = 0; i + 1 < c.n_stages; ++i) {
+            Cs /= 2;
+            any = any || (h->stage_tc[i] && !h->stage_fused[i] && h->ups_tc[i + 1] && amp_gemm_split_fusable(Cs));
+        }
+        h->ms_on = any;
+    }
+    const int n_pairs = c.n_resblocks + (h->ms_on ? 1 : 0);
+    const long long total = n_in + n_pre + nbuf * h->stage_cap + n_lat + n_wav + 64 + 2 * n_pairs * n_a;
     h->abytes = (size_t)total * sizeof(float);
     // both device allocations before any device work, so that a failed one leaves nothing behind
     // but what fail() releases
@@ -941,7 +970,7 @@ mh3a_status mh3a_create_with_allocator(const mh3a_config* cfg, const mh3a_tensor
     for (int j = 0; j < c.n_resblocks; ++j) { h->T[j] = p; p += h->stage_cap; }
     h->lat_io = p; p += n_lat;
     h->wav_io = p; p += n_wav;
-    for (int j = 0; j < c.n_resblocks && n_a > 0; ++j) {
+    for (int j = 0; j < n_pairs && n_a > 0; ++j) {
         h->A_hi[j] = p; p += n_a;
         h->A_lo[j] = p; p += n_a;
     }

@@ -457,6 +457,15 @@ struct GemmParams {
     int tpu;              // tap units per weight bulk copy (set by the launcher)
     int* err;
     int* sched;           // [next tile, CTAs done]: zero before a launch, left zero after it
+    // Fused input split of the next upsampler (R == 1, three jobs = the stage's residual blocks;
+    // ms_hi null: off).  See mean_split_rows.
+    uint8_t* ms_hi;       // [B, Cout/8, ms_Lpad] rows of 16 bytes (heads), pad ms_padl rows
+    uint8_t* ms_lo;       // tails
+    long long ms_Lpad;
+    int ms_padl;
+    int ms_blk[MH3A_MAX_RESBLOCKS];   // residual block of job z
+    int ms_z[3];                      // job of block j
+    const float* ms_x[3];             // the blocks' outputs, in block order
 };
 
 // ----------------------------------------------------------------------------------------------
@@ -532,6 +541,62 @@ __device__ __forceinline__ void add_res_group(float (&acc)[N], const float (&rq)
 #pragma unroll
             for (int c = 0; c < GW; ++c) asm volatile("add.rn.f32 %0, %0, %1;" : "+f"(acc[GW * gg + c]) : "f"(rq[c]));
         }
+    }
+}
+
+// The fused input split of the next upsampler.  In the last layer of an AMP stage the three
+// jobs are the residual blocks; the scheduler then hands out units of three tiles -- the same
+// item, rows and channels for blocks 0, 1 and 2, in that order -- so that one CTA, and in it
+// the same epilogue thread, stores all three outputs of each of its rows and columns.  At the
+// block-2 tile that thread forms the stage output -- the mean ((x0 + x1) + x2) / 3 in block
+// order, the arithmetic of the standalone split (k_split_rows), from its own two earlier stores
+// and its registers -- and writes it as head/tail rows of 8 channels into the upsampler's A
+// operand.  The threads that hold the sequence's first and last rows also zero the kMsZeroRows
+// rows before and after it, which the upsampler's window reads (its taps reach one row to
+// either side).
+constexpr int kMsZeroRows = 8;
+// Epilogue warps of at most this many columns run it (the 16- to 64-channel stages); wider
+// warps would spill (their stage keeps the standalone split).
+constexpr int kMsMaxCW = 32;
+
+template <int CW>
+__device__ __forceinline__ void mean_split_rows(const GemmParams& p, int b, int t, int o_base, long long idx0,
+                                                const float (&acc)[CW]) {
+    const int L = p.L, ngroups = p.Cout / 8;
+    uint4* hi = reinterpret_cast<uint4*>(p.ms_hi);
+    uint4* lo = reinterpret_cast<uint4*>(p.ms_lo);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int gq = 0; gq < CW / 8; ++gq) {
+        const int g = o_base / 8 + gq;
+        if (g >= ngroups) continue;   // 16-wide tiles past Cout
+        const long long rbase = ((long long)b * ngroups + g) * p.ms_Lpad + p.ms_padl;
+        if (t < L) {
+            float v[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const long long off = idx0 + (long long)(gq * 8 + c) * L;
+                const float x0 = __ldcg(p.ms_x[0] + off), x1 = __ldcg(p.ms_x[1] + off);
+                v[c] = (x0 + x1 + acc[gq * 8 + c]) * (1.0f / 3.0f);
+            }
+            uint4 hv, lv;
+            actm::split2(v[0], v[1], &hv.x, &lv.x);
+            actm::split2(v[2], v[3], &hv.y, &lv.y);
+            actm::split2(v[4], v[5], &hv.z, &lv.z);
+            actm::split2(v[6], v[7], &hv.w, &lv.w);
+            hi[rbase + t] = hv;
+            lo[rbase + t] = lv;
+        }
+        if (t == 0)
+            for (int r = 1; r <= kMsZeroRows; ++r) {
+                hi[rbase - r] = zero;
+                lo[rbase - r] = zero;
+            }
+        if (t == L - 1)
+            for (int r = 0; r < kMsZeroRows; ++r) {
+                hi[rbase + L + r] = zero;
+                lo[rbase + L + r] = zero;
+            }
     }
 }
 
@@ -726,10 +791,18 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
             bool ok = *abort_flag == 0;
             int ia = 0, ib = 0;
             bool drained = false;   // the scheduler handed this CTA its end marker
+            int unit = 0;
             for (int i = 0; ok; ++i) {
-                // dynamic schedule: tiles go out heaviest job first, each to the CTA that asks next
-                int k = atomicAdd(p.sched, 1);
-                if (k >= sc.ntiles) k = -1;
+                // dynamic schedule: tiles go out heaviest job first, each to the CTA that asks
+                // next; with the fused split, units of the three blocks' tiles in block order
+                int k;
+                if (R == 1 && p.ms_hi != nullptr) {
+                    if (i % 3 == 0) unit = atomicAdd(p.sched, 1);
+                    k = unit < sc.per_job ? p.ms_z[i % 3] * sc.per_job + unit : -1;
+                } else {
+                    k = atomicAdd(p.sched, 1);
+                    if (k >= sc.ntiles) k = -1;
+                }
                 tile_q[i % PS_TQ] = k;
                 ptx::mbar_arrive(&tile_full[i % PS_TQ]);
                 if (k < 0) {
@@ -932,6 +1005,11 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     for (int ph = 0; ph < R; ++ph) J.out[idx0 + (long long)c * Lout + ph] = acc[ph * CW + c];
                 }
             }
+            if constexpr (R == 1 && CW <= kMsMaxCW) {
+                // the block-2 tile of a unit: this thread stored blocks 0 and 1 of these rows
+                // and columns in the unit's two previous tiles
+                if (p.ms_hi != nullptr && p.ms_blk[T.z] == 2) mean_split_rows<CW>(p, T.b, t, o_base, idx0, acc);
+            }
             __syncwarp();   // the bias slice is rewritten for the next tile
         }
         if (!ok) {
@@ -1074,6 +1152,20 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     sc.n_ot = (p.Cout + NT - 1) / NT;
     sc.per_job = p.B * p.tiles_t * sc.n_ot;
     sc.ntiles = njobs * sc.per_job;
+    if (p.ms_hi) {
+        // the fused split: the three residual blocks of an AMP layer, one counter per (tile of
+        // a job, epilogue warp), whole 8-channel groups, warps narrow enough to run it
+        if (R != 1 || njobs != 3 || 4 * MT * NT / EW > kMsMaxCW || !p.ms_lo || p.Cout % 8 != 0 ||
+            p.ms_padl < kMsZeroRows || p.ms_Lpad < (long long)p.ms_padl + p.L + kMsZeroRows)
+            return -1;
+        int seen = 0;
+        for (int z = 0; z < 3; ++z) {
+            if (p.ms_blk[z] < 0 || p.ms_blk[z] > 2 || !p.ms_x[z]) return -1;
+            seen |= 1 << p.ms_blk[z];
+            p.ms_z[p.ms_blk[z]] = z;
+        }
+        if (seen != 7) return -1;
+    }
     // Passes of 8 MMA K-steps (4 taps of 32 channels) at the widest tiles; 16 K-steps (8 taps)
     // for the 32- to 128-channel convs and 16 taps of the 16-channel chunks, where fewer
     // accumulator drains measured 1-3 us per launch faster; the upsampler's pass is one whole
@@ -1246,6 +1338,12 @@ TcJob make_job(const ConvJob& J, const TcConv& tw) {
 
 }  // namespace
 
+// The 32- and 16-channel stages: their last layers have 626 units of three tiles at the bench
+// workload (B = 2), and the fused split saves its launch (ups5 35.8 -> 20.5 us, ups6 37.9 -> 24.6)
+// for 7-10 us more in the layer.  At 64 channels the 314 units leave a heavy last wave on 148
+// SMs (amp3 +22 us against ups4 -13 us), so that stage keeps the standalone split.
+bool amp_gemm_split_fusable(int C) { return C == 32 || C == 16; }
+
 bool tc_stage_supported(int C, const mh3a_config& c) {
     if (C != 512 && C != 256 && C != 128 && C != 64 && C != 32 && C != 16 && C != 8) return false;
     if (c.n_resblocks != 3) return false;
@@ -1327,8 +1425,16 @@ int launch_conv_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int
 
 int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w, int m, int half,
                        const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
-                       cudaStream_t s, int* err, int* sched) {
+                       cudaStream_t s, int* err, int* sched, const MeanSplitTarget* ms) {
     GemmParams p{};
+    if (ms) {
+        p.ms_hi = static_cast<uint8_t*>(ms->a_hi);
+        p.ms_lo = static_cast<uint8_t*>(ms->a_lo);
+        p.ms_Lpad = ms->Lpad;
+        p.ms_padl = ms->pad_l;
+        if (njobs != 3) return -1;
+        for (int j = 0; j < 3; ++j) p.ms_x[j] = cp.job[j].out;
+    }
     p.sched = sched;
     p.Cin = cp.Cin;
     p.Cout = cp.Cout;
@@ -1345,6 +1451,7 @@ int launch_amp_gemm_tc(const ConvParams& cp, int njobs, const TcStageWeights& w,
         const int j = order[z];
         const TcConv& tw = w.conv[j][m][half];
         if (!tw.dev) return -1;
+        p.ms_blk[z] = j;
         GemmJob& G = p.job[z];
         G.a_hi = static_cast<const uint8_t*>(a_hi[j]);
         G.a_lo = static_cast<const uint8_t*>(a_lo[j]);

@@ -73,9 +73,22 @@ int launch_conv_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int 
 // written by launch_act_split into a_hi[j] / a_lo[j] with pad_l zero rows before the sequence
 // and Lpad rows per (item, channel group).  `sched` points to two device ints, zero before the
 // launch (the kernel leaves them zero when it completes): the dynamic tile scheduler's state.
+// With `ms` (the last layer of a stage whose next upsampler runs on the tensor cores; three
+// residual blocks), the kernel also writes the stage output -- the mean of the blocks' outputs
+// -- as that upsampler's head/tail rows (the standalone split's arithmetic, bit for bit), with
+// the zero rows its window reads next to the sequence.
+// Whether the AMP GEMM at C channels takes a MeanSplitTarget (the 16- and 32-channel stages;
+// the kernel itself accepts epilogue warps of at most 32 columns).
+bool amp_gemm_split_fusable(int C);
+struct MeanSplitTarget {
+    void* a_hi;           // [B, C/8, Lpad] rows of 8 bf16 heads; must not be an operand of this launch
+    void* a_lo;           // tails
+    int pad_l;            // rows before the sequence (at least 8)
+    long long Lpad;       // rows per (item, channel group), at least pad_l + L + 8
+};
 int launch_amp_gemm_tc(const ConvParams& p, int njobs, const TcStageWeights& w, int m, int half,
                        const void* const* a_hi, const void* const* a_lo, int pad_l, long long Lpad,
-                       cudaStream_t s, int* err, int* sched);
+                       cudaStream_t s, int* err, int* sched, const MeanSplitTarget* ms = nullptr);
 
 // conv_pre and the upsamplers on the persistent GEMM, reading their input as pre-split rows
 // (launch_split_rows) with pad_l zero rows before the sequence and Lpad rows per channel group.
