@@ -63,6 +63,22 @@ def test_replay_matches_direct_decode_and_counts_the_same_kernels(decs):
     graph.check_device_error()
 
 
+def test_decode_kernel_count(decs):
+    """The launches of one BF16X3 decode at the default architecture: the fused projection and
+    conv_pre (2); seven upsamplers, five of them after a standalone input split (12: the last
+    layers of the 32- and 16-channel stages write upsamplers 5 and 6's operands themselves);
+    six AMP stages of six layers, each an activation and a GEMM (72); the fused 8-channel stage
+    and the fused tail (2)."""
+    arch, eager, _ = decs
+    z = _lat(arch, 1, 6, 43)
+    eager.decode(z)
+    torch.cuda.synchronize()
+    n0 = eager.launch_count()
+    eager.decode(z)
+    torch.cuda.synchronize()
+    assert eager.launch_count() - n0 == 2 + 12 + 72 + 2
+
+
 def test_several_shapes_and_slot_replacement(decs):
     arch, eager, graph = decs
     s = torch.cuda.Stream()
