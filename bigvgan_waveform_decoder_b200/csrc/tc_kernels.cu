@@ -1546,7 +1546,10 @@ int launch_convT_gemm(const ConvTParams& q, const TcStageWeights& w, const void*
     if (q.r == 5 && NT == 32) return launch_gemm_ps<1, 32, 4, 8, 5>(p, 1, s);
     if (q.r == 2) {
         switch (NT) {
-            case 64: return launch_gemm_ps<2, 64, 4, 8, 2>(p, 1, s);
+            // 128-row tiles at 64 output channels: upsamplers 2 and 3 have 158-160 tiles of 256
+            // rows at the bench workload, 1.08 waves on 148 SMs; 128-row tiles measured 58.3 ->
+            // 56.4 and 42.0 -> 40.0 us per launch
+            case 64: return launch_gemm_ps<1, 64, 4, 8, 2>(p, 1, s);
             case 32: return launch_gemm_ps<2, 32, 4, 8, 2>(p, 1, s);
             case 16: return launch_gemm_ps<2, 16, 4, 8, 2>(p, 1, s);
             default: return -1;
