@@ -49,7 +49,7 @@ METRIC = "decoded audio-seconds/sec at 32 kHz on 1 B200; % of roofline per stage
 # Tile shape <MT, NT, KGT, EW, R> of the persistent GEMM per AMP width (as dispatched by the
 # library), for labelling the roofline's kernel.
 GEMM_TILE = {512: "1, 256, 4, 8, 1", 256: "1, 256, 4, 8, 1", 128: "2, 128, 4, 8, 1",
-             64: "2, 64, 4, 16, 1", 32: "2, 32, 4, 16, 1", 16: "4, 16, 2, 16, 1", 8: "4, 16, 1, 16, 1"}
+             64: "2, 64, 4, 16, 1", 32: "2, 32, 4, 8, 1", 16: "2, 16, 2, 8, 1", 8: "4, 16, 1, 16, 1"}
 # DRAM bytes (read + write) per launch of that GEMM kernel on this workload, keyed by (channels,
 # B * N), from one ncu capture (profiles/k_gemm_ps_stage1_B2_L10000.md); null when unmeasured
 # or when the kernel changed after the capture.

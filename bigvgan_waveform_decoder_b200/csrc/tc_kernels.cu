@@ -482,7 +482,7 @@ constexpr int ps_threads(int EW) { return 64 + 32 * EW; }
 constexpr int PS_MAXS = 8;                              // ring stages (max)
 constexpr int PS_TQ = 16;                               // tile-index queue entries
 constexpr int PS_BAR_BYTES = 8 * (4 * PS_MAXS + 5 + PS_TQ) + 8 + 4 * PS_TQ;   // barriers, flags, queue
-constexpr int PS_BUFCOLS = 256;                         // TMEM columns per accumulator buffer
+constexpr int PS_BUFCOLS = 256;                         // TMEM columns per accumulator buffer (max)
 
 struct PsPlan {
     int RS;             // window rows per channel group (max over jobs)
@@ -612,13 +612,31 @@ __device__ __forceinline__ void mean_split_rows(const GemmParams& p, int b, int 
 // all R phases (zero rows where the group has no tap), so one MMA of N = R NT covers every
 // phase region and the group's first unit initialises all of them.  A pass is
 // then one whole chunk, so that the first tap of every phase (j < R) starts its region.
+// Accumulator columns per M tile, TMEM columns per buffer, and CTAs per SM.  A GEMM with 8
+// epilogue warps whose accumulators take at most 128 columns per buffer (the 16- and 32-channel
+// AMP convs, the rate-2 upsamplers) runs two CTAs per SM: their double buffers fill the 512
+// TMEM columns exactly, their threads the register file, and each takes at most half the
+// shared memory (so no third CTA, of this launch or the next, can wait on tensor memory).
+// Measured per launch against one CTA per SM: AMP 32 channels 48.1 -> 41.9 us, 16 channels
+// 49.9 -> 45.0 us (with 16 epilogue warps there); upsamplers 2-6 56 -> 50, 40 -> 38, 36 -> 34,
+// 21 -> 18, 25 -> 19 us.
+__host__ __device__ constexpr int ps_rstr(int NT, int R) { return interleaved_b(NT, R) ? 2 * NT : R * NT; }
+__host__ __device__ constexpr int ps_ctas(int MT, int NT, int EW, int R) {
+    return (EW == 8 && MT * ps_rstr(NT, R) <= 128) ? 2 : 1;
+}
+__host__ __device__ constexpr int ps_bufcols(int MT, int NT, int EW, int R) {
+    return ps_ctas(MT, NT, EW, R) == 2 ? 128 : PS_BUFCOLS;
+}
+
 template <int MT, int NT, int KGT, int EW, int R>
-__global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
+__global__ void __launch_bounds__(ps_threads(EW), ps_ctas(MT, NT, EW, R))
+    k_gemm_ps(const GemmParams p, const PsSched sc, const PsPlan pl) {
     extern __shared__ __align__(1024) uint8_t smem[];
     ptx::grid_dep_wait();   // launched as a programmatic dependent (see launch_dependent)
     constexpr bool ILV = interleaved_b(NT, R);            // two-MMA K-steps, head | cross columns
     constexpr int RSTR = ILV ? 2 * NT : R * NT;            // accumulator columns per M tile
-    static_assert(MT * RSTR <= PS_BUFCOLS, "one accumulator buffer holds MT x RSTR columns");
+    constexpr int BUFC = ps_bufcols(MT, NT, EW, R);        // TMEM columns per accumulator buffer
+    static_assert(MT * RSTR <= BUFC, "one accumulator buffer holds MT x RSTR columns");
     static_assert(R == 1 || KGT >= 2, "the upsampler uses 16- or 32-channel chunks");
     static_assert(KGT == 1 || KGT == 2 || KGT == 4, "channel groups per chunk");
     static_assert(EW == 8 || EW == 16, "epilogue warps");
@@ -669,7 +687,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
-        ptx::tmem_alloc(tmem_slot, 2 * PS_BUFCOLS);
+        ptx::tmem_alloc(tmem_slot, 2 * BUFC);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -723,7 +741,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
                     // KGT >= 2: unit = tap, K-steps over channel-group pairs.  KGT == 1: unit =
                     // tap pair, one K-step whose two core-matrix columns are taps 2u and 2u+1.
                     const uint32_t bh = bh0 + (uint32_t)ucopy * (TAPB >> 4);
-                    uint32_t dbase = tmem + (uint32_t)(buf * PS_BUFCOLS);
+                    uint32_t dbase = tmem + (uint32_t)(buf * BUFC);
                     uint32_t arow = ashift;
                     bool first = upass == 0;
                     if (GRP) {
@@ -951,7 +969,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
 #pragma unroll
                         for (int cb = 0; cb < CW; cb += 8) {
                             float v[8];
-                            ptx::tmem_ld8(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
+                            ptx::tmem_ld8(lane_addr + (uint32_t)(buf * BUFC + ph * NT + cb), v);
 #pragma unroll
                             for (int c = 0; c < 8; ++c) acc[ph * CW + cb + c] += v[c];
                         }
@@ -959,10 +977,10 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
 #pragma unroll
                         for (int cb = 0; cb < CW; cb += 16) {
                             float v[16];
-                            ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + ph * NT + cb), v);
+                            ptx::tmem_ld16(lane_addr + (uint32_t)(buf * BUFC + ph * NT + cb), v);
                             if (ILV) {
                                 float x[16];
-                                ptx::tmem_ld16(lane_addr + (uint32_t)(buf * PS_BUFCOLS + NT + cb), x);
+                                ptx::tmem_ld16(lane_addr + (uint32_t)(buf * BUFC + NT + cb), x);
 #pragma unroll
                                 for (int c = 0; c < 16; ++c) v[c] += x[c];
                             }
@@ -1021,7 +1039,7 @@ __global__ void __launch_bounds__(ps_threads(EW), 1) k_gemm_ps(const GemmParams 
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 0) ptx::tmem_dealloc(tmem, 2 * PS_BUFCOLS);
+    if (warp == 0) ptx::tmem_dealloc(tmem, 2 * BUFC);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -1146,7 +1164,8 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     // 51 -> 49 us; upsamplers 1024 -> 512 channels 66.5 -> 60.5 us, 512 -> 256 70.7 -> 64.5 us,
     // 256 -> 128 60.4 -> 58.3 us; 32 KB copies gained only the last).  The widest AMP tiles and
     // the narrow 2-group chunks stay at 16 KB, where larger copies measured slower or equal.
-    const int wbytes = (R > 1 || (KGT == 4 && NT <= 128)) ? 65536 : 16384;
+    constexpr int CTAS = ps_ctas(MT, NT, EW, R);
+    const int wbytes = (CTAS == 1 && (R > 1 || (KGT == 4 && NT <= 128))) ? 65536 : 16384;
     p.tpu = std::max(1, std::min(kumax, wbytes / TAPB));
     PsSched sc{};
     sc.n_ot = (p.Cout + NT - 1) / NT;
@@ -1176,7 +1195,7 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     pl.SA = 2 * KGT * pl.RS * 16;
     pl.SB = p.tpu * TAPB;
     constexpr int kBarBytes = PS_BAR_BYTES + 4 * EW * 4 * MT * NT / EW;   // + the epilogue's bias slices
-    constexpr int kBudget = 227 * 1024 - kBarBytes - 64;
+    constexpr int kBudget = (CTAS == 2 ? 113 * 1024 : 227 * 1024) - kBarBytes - 64;
     pl.nsa = (4 * pl.SA <= kBudget / 2) ? 4 : 3;
     if (pl.nsa * pl.SA + 2 * pl.SB > kBudget) pl.nsa = 2;
     pl.nsb = std::min(PS_MAXS, (kBudget - pl.nsa * pl.SA) / pl.SB);
@@ -1184,15 +1203,15 @@ int launch_gemm_ps(const GemmParams& p0, int njobs, cudaStream_t s) {
     pl.offB = pl.nsa * pl.SA;
     pl.offBar = (pl.offB + pl.nsb * pl.SB + 15) / 16 * 16;
     pl.smem = pl.offBar + kBarBytes;
-    // at least half the SM's shared memory, so that a second CTA never waits on the first's
-    // tensor memory
-    const int smem_req = std::max(pl.smem, 116 * 1024);
-    if (smem_req > 227 * 1024) return -1;
+    // One CTA per SM takes at least half the SM's shared memory, so that a second CTA never
+    // waits on the first's tensor memory; two take at most half each.
+    const int smem_req = CTAS == 2 ? pl.smem : std::max(pl.smem, 116 * 1024);
+    if (smem_req > (CTAS == 2 ? 113 : 227) * 1024) return -1;
     const int nsm = sm_count();
     if (nsm <= 0) return -1;
     auto kern = k_gemm_ps<MT, NT, KGT, EW, R>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_req) != cudaSuccess) return -1;
-    const int grid = std::min(sc.ntiles, nsm);
+    const int grid = std::min(sc.ntiles, CTAS * nsm);
     return launch_dependent(kern, dim3(grid), dim3(ps_threads(EW)), smem_req, s, p, sc, pl) == cudaSuccess ? 1 : -1;
 }
 
@@ -1202,8 +1221,9 @@ int dispatch_gemm(const GemmParams& p, int njobs, cudaStream_t s) {
         case 256: return launch_gemm_ps<1, 256, 4, 8, 1>(p, njobs, s);
         case 128: return launch_gemm_ps<2, 128, 4, 8, 1>(p, njobs, s);
         case 64: return launch_gemm_ps<2, 64, 4, 16, 1>(p, njobs, s);
-        case 32: return launch_gemm_ps<2, 32, 4, 16, 1>(p, njobs, s);
-        case 16: return launch_gemm_ps<4, 16, 2, 16, 1>(p, njobs, s);
+        // two CTAs per SM at 32 and 16 channels (see ps_ctas)
+        case 32: return launch_gemm_ps<2, 32, 4, 8, 1>(p, njobs, s);
+        case 16: return launch_gemm_ps<2, 16, 2, 8, 1>(p, njobs, s);
         case 8: return launch_gemm_ps<4, 16, 1, 16, 1>(p, njobs, s);
         default: return -1;
     }
