@@ -1360,8 +1360,9 @@ TcJob make_job(const ConvJob& J, const TcConv& tw) {
 
 // The 32- and 16-channel stages: their last layers have 626 units of three tiles at the bench
 // workload (B = 2), and the fused split saves its launch (ups5 35.8 -> 20.5 us, ups6 37.9 -> 24.6)
-// for 7-10 us more in the layer.  At 64 channels the 314 units leave a heavy last wave on 148
-// SMs (amp3 +22 us against ups4 -13 us), so that stage keeps the standalone split.
+// for 7-10 us more in the layer (with two CTAs per SM: stages 4-5 and upsamplers 5-6 872 us
+// against 887 us with the standalone split).  At 64 channels the 314 units leave a heavy last
+// wave on 148 SMs (amp3 +22 us against ups4 -13 us), so that stage keeps the standalone split.
 bool amp_gemm_split_fusable(int C) { return C == 32 || C == 16; }
 
 bool tc_stage_supported(int C, const mh3a_config& c) {
