@@ -7,6 +7,8 @@ against the stage-1 figure bench.py reports per GEMM launch (55.05 GFLOP).
 """
 from __future__ import annotations
 
+import os
+
 import pytest
 
 from bigvgan_waveform_decoder_b200 import perfmodel as PM
@@ -74,3 +76,20 @@ def test_roofline_time_takes_the_slowest_pipe():
 
 def test_fp32_peak_from_unit_counts():
     assert PM.fp32_peak_tflops(1965.0) == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
+
+
+def test_bench_launches_directly_under_a_profiler(monkeypatch):
+    """bench.py replays decodes from CUDA graphs unless a profiler has injected itself into the
+    CUDA runtime (Nsight Compute sets its transport variables in the program it starts)."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    for k in bench.PROFILER_ENV:
+        monkeypatch.delenv(k, raising=False)
+    assert bench.graphs_allowed()
+    for k in bench.PROFILER_ENV:
+        monkeypatch.setenv(k, "1")
+        assert not bench.graphs_allowed(), k
+        monkeypatch.delenv(k)
+    assert bench.graphs_allowed()
